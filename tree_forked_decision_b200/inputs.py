@@ -1,0 +1,243 @@
+"""Seeded synthetic inputs: decision trees and layer tensors.
+
+This module only draws random numbers and lays them out; it holds none of the
+method's arithmetic.  Both the CUDA path and the CPU oracle consume exactly the
+tensors it returns.
+
+Tree shapes follow the workloads: a shared prefix (the root node) plus option
+branches laid out in one flattened token stream (kongchang.com, introduction
+and "ForkAttention" section); up to 256 options per request (techfi24.com,
+"Performances et comparaison"); resumed requests carry checkpointed history
+(kongchang.com, "ForkAttention" section).  Value distributions: q, k, v ~
+N(0, 1); for Gated DeltaNet, q and k are L2-normalised per head, the gate is
+passed as g = log(alpha) = -scale * softplus(x), x ~ N(0, 1), and
+beta = sigmoid(N(0, 1)).
+
+Stream order: requests in order; within a request, nodes in index order with
+parent[i] < i; node 0 of every request is its root.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass
+class Tree:
+    req_node_ptr: np.ndarray  # int32 [R+1]
+    parent: np.ndarray        # int32 [N], request-local parent, -1 for a root
+    seg_len: np.ndarray       # int32 [N], tokens per node in stream order
+    past_len: np.ndarray      # int32 [R], checkpointed tokens before the root
+    levels: int               # branch levels below the root (by construction)
+
+    @property
+    def R(self) -> int:
+        return len(self.req_node_ptr) - 1
+
+    @property
+    def N(self) -> int:
+        return int(self.req_node_ptr[-1])
+
+    @property
+    def T(self) -> int:
+        return int(self.seg_len.sum())
+
+    @property
+    def P_past(self) -> int:
+        return int(self.past_len.sum())
+
+    @property
+    def root_tokens(self) -> int:
+        roots = self.req_node_ptr[:-1][self.req_node_ptr[:-1] < self.req_node_ptr[1:]]
+        return int(self.seg_len[roots].sum())
+
+    @property
+    def branch_tokens(self) -> int:
+        return self.T - self.root_tokens
+
+    def arrays(self):
+        return self.req_node_ptr, self.parent, self.seg_len, self.past_len
+
+
+def _tree(reqs, levels):
+    """reqs: list of (past_len, [(parent_local, seg_len), ...])."""
+    rp = [0]
+    parent, seg, past = [], [], []
+    for p_len, nodes in reqs:
+        past.append(p_len)
+        for pa, sl in nodes:
+            parent.append(pa)
+            seg.append(sl)
+        rp.append(rp[-1] + len(nodes))
+    return Tree(np.asarray(rp, np.int32), np.asarray(parent, np.int32),
+                np.asarray(seg, np.int32), np.asarray(past, np.int32), levels)
+
+
+def fanout_tree(R: int, prefix: int, branches: int, branch_len: int,
+                past: int = 0) -> Tree:
+    """R requests, each a root of `prefix` tokens and `branches` leaves of
+    `branch_len` tokens (depth 1)."""
+    nodes = [(-1, prefix)] + [(0, branch_len)] * branches
+    return _tree([(past, nodes)] * R, 1 if branches else 0)
+
+
+def leveled_tree(rng: np.random.Generator, R: int, depth_range=(1, 3),
+                 options_range=(2, 256), prefix_range=(256, 8192),
+                 branch_range=(4, 64), n_resume: int = 0,
+                 resume_delta=(4, 64)) -> Tree:
+    """Mixed batch of level-structured trees.
+
+    Per request: D ~ U{depth_range}, O ~ U{options_range} leaves, prefix
+    P ~ U{prefix_range}, every non-root segment ~ U{branch_range}.  Level sizes
+    n_0 = 1, n_k = ceil(O^(k/D)) for 0 < k < D, n_D = O; node j of level k hangs
+    under node (j mod n_{k-1}) of level k-1.  `n_resume` requests (seeded
+    choice) resume from a checkpoint holding their first P - delta prefix
+    tokens, delta ~ U{resume_delta}: those tokens become past, the root keeps
+    delta tokens.
+    """
+    reqs = []
+    max_levels = 0
+    resumed = set(rng.choice(R, size=n_resume, replace=False).tolist()) if n_resume else set()
+    for r in range(R):
+        D = int(rng.integers(depth_range[0], depth_range[1] + 1))
+        O = int(rng.integers(options_range[0], options_range[1] + 1))
+        P = int(rng.integers(prefix_range[0], prefix_range[1] + 1))
+        sizes = [1] + [int(math.ceil(O ** (k / D))) for k in range(1, D)] + [O]
+        first = [0]
+        for s in sizes[:-1]:
+            first.append(first[-1] + s)
+        nodes = []
+        for k, nk in enumerate(sizes):
+            for j in range(nk):
+                if k == 0:
+                    nodes.append([-1, P])
+                else:
+                    pa = first[k - 1] + (j % sizes[k - 1])
+                    nodes.append([pa, int(rng.integers(branch_range[0], branch_range[1] + 1))])
+        past = 0
+        if r in resumed:
+            delta = int(rng.integers(resume_delta[0], resume_delta[1] + 1))
+            delta = min(delta, P)
+            past = P - delta
+            nodes[0][1] = delta
+        max_levels = max(max_levels, D)
+        reqs.append((past, [tuple(x) for x in nodes]))
+    return _tree(reqs, max_levels)
+
+
+def random_tree(rng: np.random.Generator, R: int, max_nodes: int = 8,
+                prefix_range=(0, 40), branch_range=(1, 9),
+                past_range=(0, 0)) -> Tree:
+    """Small irregular trees for tests: each node's parent is uniform among the
+    earlier nodes of its request."""
+    reqs = []
+    levels = 0
+    for _ in range(R):
+        n = int(rng.integers(1, max_nodes + 1))
+        nodes = [(-1, int(rng.integers(prefix_range[0], prefix_range[1] + 1)))]
+        depth = [0]
+        for i in range(1, n):
+            pa = int(rng.integers(0, i))
+            nodes.append((pa, int(rng.integers(branch_range[0], branch_range[1] + 1))))
+            depth.append(depth[pa] + 1)
+        levels = max(levels, max(depth))
+        reqs.append((int(rng.integers(past_range[0], past_range[1] + 1)), nodes))
+    return _tree(reqs, levels)
+
+
+def _to(x: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x)).to(dtype)
+
+
+def attn_inputs(tree: Tree, Hq: int, Hkv: int, d: int, dtype: torch.dtype,
+                rng: np.random.Generator):
+    """q [T,Hq,d], k,v [T,Hkv,d], past_k,past_v [sum(past),Hkv,d]; N(0,1)."""
+    T, P = tree.T, tree.P_past
+    q = rng.standard_normal((T, Hq, d), dtype=np.float32)
+    k = rng.standard_normal((T, Hkv, d), dtype=np.float32)
+    v = rng.standard_normal((T, Hkv, d), dtype=np.float32)
+    pk = rng.standard_normal((P, Hkv, d), dtype=np.float32)
+    pv = rng.standard_normal((P, Hkv, d), dtype=np.float32)
+    return dict(q=_to(q, dtype), k=_to(k, dtype), v=_to(v, dtype),
+                past_k=_to(pk, dtype), past_v=_to(pv, dtype))
+
+
+def _l2n(x: np.ndarray) -> np.ndarray:
+    n = np.sqrt((x.astype(np.float32) ** 2).sum(-1, keepdims=True, dtype=np.float32))
+    return (x / np.maximum(n, np.float32(1e-6))).astype(np.float32)
+
+
+def gdn_inputs(tree: Tree, H: int, dk: int, dv: int, dtype: torch.dtype,
+               rng: np.random.Generator, gate_scale: float = 1.0,
+               state_scale: float = 0.1):
+    """q,k [T,H,dk] (L2-normalised), v [T,H,dv], g = -gate_scale*softplus(x)
+    and beta = sigmoid(y) [T,H] float32 with x, y ~ N(0,1); state_in
+    [R,H,dv,dk] float32: N(0, state_scale^2) for requests with past history,
+    zero otherwise."""
+    T, R = tree.T, tree.R
+    q = _l2n(rng.standard_normal((T, H, dk), dtype=np.float32))
+    k = _l2n(rng.standard_normal((T, H, dk), dtype=np.float32))
+    v = rng.standard_normal((T, H, dv), dtype=np.float32)
+    x = rng.standard_normal((T, H)).astype(np.float64)
+    g = (-gate_scale * np.logaddexp(0.0, x)).astype(np.float32)
+    y = rng.standard_normal((T, H)).astype(np.float64)
+    beta = (1.0 / (1.0 + np.exp(-y))).astype(np.float32)
+    state = np.zeros((R, H, dv, dk), np.float32)
+    for r in range(R):
+        if tree.past_len[r] > 0:
+            state[r] = rng.standard_normal((H, dv, dk), dtype=np.float32) * np.float32(state_scale)
+    return dict(q=_to(q, dtype), k=_to(k, dtype), v=_to(v, dtype),
+                g=torch.from_numpy(g), beta=torch.from_numpy(beta),
+                state_in=torch.from_numpy(state))
+
+
+# ---------------------------------------------------------------------------
+# Named workloads.  Each returns (tree, attention spec or None, GDN spec or
+# None, dtype).  seed defaults to the workload's index.
+# ---------------------------------------------------------------------------
+
+WORKLOADS = {
+    "tiny_fp32": dict(idx=1, desc="1 request, prefix 64, 4 branches x 8, attn 4 heads d=64, GDN 4 heads dk=dv=64, fp32"),
+    "attn_fanout_bf16": dict(idx=2, desc="8 requests, prefix 2048, 16 branches x 32, GQA Hq=16 Hkv=4 d=128, bf16"),
+    "gdn_fanout_bf16": dict(idx=3, desc="8 requests, prefix 4096, 64 branches x 16, GDN 16 heads dk=dv=128, bf16"),
+    "mixed_hybrid_bf16": dict(idx=4, desc="32 requests depth 1-3, 2-256 options, prefix 256-8192, branches 4-64, half resumed; attn Hq=16 Hkv=4 d=128 + GDN 16x128, bf16"),
+    "large_fanout_bf16": dict(idx=5, desc="4 requests, prefix 32768, 256 branches x 8, attn Hq=32 Hkv=8 d=128 + GDN 32 heads dk=dv=128, bf16"),
+}
+
+
+def workload(name: str, seed: int | None = None):
+    spec = WORKLOADS[name]
+    rng = np.random.default_rng(spec["idx"] if seed is None else seed)
+    if name == "tiny_fp32":
+        tree = fanout_tree(1, 64, 4, 8)
+        return tree, dict(Hq=4, Hkv=4, d=64), dict(H=4, dk=64, dv=64, gate_scale=1.0), torch.float32, rng
+    if name == "attn_fanout_bf16":
+        tree = fanout_tree(8, 2048, 16, 32)
+        return tree, dict(Hq=16, Hkv=4, d=128), None, torch.bfloat16, rng
+    if name == "gdn_fanout_bf16":
+        tree = fanout_tree(8, 4096, 64, 16)
+        return tree, None, dict(H=16, dk=128, dv=128, gate_scale=0.1), torch.bfloat16, rng
+    if name == "mixed_hybrid_bf16":
+        tree = leveled_tree(rng, 32, n_resume=16)
+        return tree, dict(Hq=16, Hkv=4, d=128), dict(H=16, dk=128, dv=128, gate_scale=0.1), torch.bfloat16, rng
+    if name == "large_fanout_bf16":
+        tree = fanout_tree(4, 32768, 256, 8)
+        return tree, dict(Hq=32, Hkv=8, d=128), dict(H=32, dk=128, dv=128, gate_scale=0.1), torch.bfloat16, rng
+    raise KeyError(name)
+
+
+def make_inputs(name: str, seed: int | None = None):
+    """Tree plus host tensors for a named workload."""
+    tree, aspec, gspec, dtype, rng = workload(name, seed)
+    attn = gdn = None
+    if aspec:
+        attn = attn_inputs(tree, aspec["Hq"], aspec["Hkv"], aspec["d"], dtype, rng)
+        attn.update(aspec)
+    if gspec:
+        gdn = gdn_inputs(tree, gspec["H"], gspec["dk"], gspec["dv"], dtype, rng,
+                         gate_scale=gspec["gate_scale"])
+        gdn.update(gspec)
+    return tree, attn, gdn, dtype
