@@ -1,0 +1,243 @@
+/*
+ * flide.h -- C ABI of libflide.so: the ForkAttention hot path on one B200.
+ *
+ * The operations follow the pages on Flide ("tree-forked decision inference"):
+ *   - a decision request is a shared prefix plus option branches, all laid out
+ *     in ONE flattened token stream, with the request's logical tree held as
+ *     GPU-resident indices (kongchang.com article, introduction and
+ *     "ForkAttention" section);
+ *   - every branch query must equal an isolated forward pass over its own
+ *     ancestors, for softmax attention and for Gated DeltaNet layers
+ *     (kongchang.com, "ForkAttention" section and Gated DeltaNet box); branch
+ *     tokens never attend to other branches (kongchang.com, attention-mask
+ *     section);
+ *   - the network state is cloned at the decision point instead of being
+ *     recomputed (techfi24.com, "Mécanisme d'Exact State Forking"), and growing
+ *     histories resume from checkpoints saved by earlier passes
+ *     (kongchang.com, "ForkAttention" section).
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers into caller-owned memory.  The
+ *     library allocates nothing and keeps no state between calls except
+ *     process-wide cached function pointers.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream), launches only kernels, and reads every data-dependent
+ *     size (actual node/token counts, tree depth, work counts) from device
+ *     memory, so a call sequence can be captured once into a CUDA graph and
+ *     replayed for any tree that fits the capacities it was captured with.
+ *   - The return value reports errors detected on the host (bad arguments,
+ *     unsupported shapes, launch failures).  Errors that depend on device data
+ *     (malformed tree, capacity overflow) are written to the index's `status`
+ *     word (first error wins); kernels that find a non-zero status do nothing.
+ *     Read it after synchronising the stream.  No call aborts the process.
+ *   - Stream layout: requests in order; within a request, nodes in index order
+ *     with parent[i] < i; node 0 of each request is its root (the shared
+ *     prefix).  Tensors are row-major [token, head, dim].
+ */
+#ifndef FLIDE_H
+#define FLIDE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define FLIDE_OK 0
+#define FLIDE_ERR_INVALID 1  /* malformed tree: parent >= self, root with parent != -1,
+                                non-root seg_len < 1, req_node_ptr not monotone   */
+#define FLIDE_ERR_SHAPE 2    /* unsupported head dim / dtype, Hq % Hkv != 0, NULL arg */
+#define FLIDE_ERR_CAPACITY 3 /* tree or data larger than the capacities given      */
+#define FLIDE_ERR_CUDA 4     /* a CUDA runtime call or kernel launch failed        */
+#define FLIDE_ERR_TIMEOUT 5  /* a bounded device-side wait expired                 */
+
+/* ---- element types ----------------------------------------------------- */
+#define FLIDE_F32 0
+#define FLIDE_BF16 1
+
+/* ---- flags for flide_fork_attn / flide_fork_gdn ------------------------ */
+#define FLIDE_FLAG_PORTABLE 1 /* force the portable SIMT kernels (any d, any dtype) */
+
+typedef void *flide_stream; /* cudaStream_t */
+
+/* Number of int32 entries in flide_tree_index.counts. */
+#define FLIDE_COUNTS 16
+/* counts[] slots written by flide_tree_build */
+#define FLIDE_CNT_N 0          /* actual nodes  = req_node_ptr[R]              */
+#define FLIDE_CNT_T 1          /* actual tokens = sum(seg_len)                 */
+#define FLIDE_CNT_PAST 2       /* packed past rows = sum(past_len)             */
+#define FLIDE_CNT_DEPTH 3      /* deepest level present (root = 0)             */
+#define FLIDE_CNT_SLOTS 4      /* node-state slots used (roots + inner nodes)  */
+#define FLIDE_CNT_BRANCH_TOK 5 /* tokens of non-root nodes                     */
+#define FLIDE_CNT_ROOT_TOK 6   /* tokens of root nodes                         */
+#define FLIDE_CNT_CKPT_ROWS 7  /* sum over requests of past_len + root seg_len */
+
+/*
+ * Tree descriptor: the request trees of one batch (kongchang.com,
+ * "ForkAttention": the logical tree of each decision request, encoded as
+ * indices).  R, N, T and max_depth are CAPACITIES (host integers); the actual
+ * sizes are read on the device: N_actual = req_node_ptr[R],
+ * T_actual = sum(seg_len[0..N_actual)).  Requests with no nodes
+ * (req_node_ptr[r] == req_node_ptr[r+1]) are allowed and act as padding.
+ */
+typedef struct {
+  int32_t R, N, T;             /* capacities: requests, nodes, stream tokens    */
+  int32_t max_depth;           /* capacity: deepest level below the root        */
+  const int32_t *req_node_ptr; /* [R+1] node ranges; req_node_ptr[0] == 0      */
+  const int32_t *parent;       /* [N] request-local parent, -1 for the root     */
+  const int32_t *seg_len;      /* [N] tokens of each node (root may be 0)       */
+  const int32_t *past_len;     /* [R] checkpointed tokens before the root       */
+} flide_tree_desc;
+
+/*
+ * Device-resident tree index, carved by flide_tree_index_init from ONE
+ * caller-allocated device buffer of flide_tree_index_bytes() bytes.  All
+ * arrays are int32 and written by flide_tree_build:
+ *   node_start[N+1]  exclusive prefix sum of seg_len (stream offset of each node)
+ *   node_req[N]      request of each node
+ *   depth[N]         edges from the request root
+ *   anc_ptr[N+1]     CSR row pointers; row n lists n's ancestors root..n
+ *   anc_node[...]    CSR entries (global node ids), N*(max_depth+1) capacity
+ *   ctx_len[N]       past_len + tokens of all ancestors and the node itself
+ *   token_node[T]    node of each stream token
+ *   token_pos[T]     position of the token in its isolated sequence
+ *                    (past_len + tokens of strict ancestors + offset in node)
+ *   past_start[R+1]  exclusive prefix sum of past_len (rows of the packed past)
+ *   req_node[R+1]    copy of req_node_ptr (first node = root of each request)
+ *   level_ptr[max_depth+2], level_node[N]  nodes grouped by depth, ascending id
+ *   state_slot[N]    slot of the node's end state in a node-state buffer, for
+ *                    roots and for nodes with children; -1 for leaves
+ *   ckpt_start[R+1]  exclusive prefix sum of past_len + root seg_len
+ *   status[1]        first device-detected error (FLIDE_* code), 0 if none
+ *   counts[FLIDE_COUNTS]  actual sizes, see FLIDE_CNT_*
+ *   work[...]        per-call scratch of the layer kernels
+ */
+typedef struct {
+  int32_t R, N, T, max_depth; /* capacities the buffer was laid out for */
+  int32_t *status, *counts;
+  int32_t *node_start, *node_req, *depth, *anc_ptr, *anc_node, *ctx_len;
+  int32_t *token_node, *token_pos, *past_start, *req_node, *level_ptr, *level_node;
+  int32_t *state_slot, *ckpt_start, *work;
+  int64_t work_len; /* int32 entries available in work */
+} flide_tree_index;
+
+/* Bytes of device memory a tree index with these capacities needs (256-byte
+ * aligned sub-arrays).  Returns 0 for negative capacities. */
+size_t flide_tree_index_bytes(int32_t R, int32_t N, int32_t T, int32_t max_depth);
+
+/* Lays out `idx` over `dev_buf` (device memory of at least `bytes` bytes,
+ * 256-byte aligned).  Host only, no device access.  Returns FLIDE_OK,
+ * FLIDE_ERR_SHAPE (NULL pointer, negative capacity, misaligned buffer) or
+ * FLIDE_ERR_CAPACITY (buffer too small). */
+int flide_tree_index_init(flide_tree_index *idx, void *dev_buf, size_t bytes,
+                          int32_t R, int32_t N, int32_t T, int32_t max_depth);
+
+/*
+ * Tree-index build (kongchang.com, "ForkAttention": topology expressed as
+ * GPU metadata).  Validates the tree and fills every array of `idx` from
+ * `desc` (whose capacities must not exceed idx's).  Resets idx->status first.
+ * Device-detected errors: FLIDE_ERR_INVALID, FLIDE_ERR_CAPACITY (more nodes,
+ * tokens or levels than the capacities).
+ */
+int flide_tree_build(const flide_tree_desc *desc, flide_tree_index *idx,
+                     flide_stream stream);
+
+/*
+ * Fork attention (kongchang.com, "ForkAttention" and attention-mask
+ * sections): every query token attends to exactly the keys of its isolated
+ * sequence -- its request's past rows, every token of its ancestors, and the
+ * tokens of its own node up to and including itself:
+ *     o = softmax(scale * q k^T) v   over those keys, fp32 accumulation.
+ * GQA: query head h reads kv head h / (Hq/Hkv).
+ *   q      [T, Hq, d]    dtype            out [T, Hq, d] dtype
+ *   k, v   [T, Hkv, d]   dtype            (T = idx->T, the token capacity)
+ *   past_k, past_v [past_rows, Hkv, d] dtype, packed in request order
+ *          (rows of request r start at idx->past_start[r]); may be NULL (with
+ *          past_rows == 0) when no request has past.  A request with past rows
+ *          and NULL past pointers sets FLIDE_ERR_SHAPE in the status word.
+ * dtype FLIDE_F32 or FLIDE_BF16.  With bf16, d == 128, 128 % (Hq/Hkv) == 0 and
+ * idx->max_depth <= 8 the tensor-core kernel runs (tcgen05 MMA, TMA, TMEM);
+ * otherwise, or with FLIDE_FLAG_PORTABLE, the portable kernel (d a multiple of
+ * 32, <= 256).
+ * Uses idx->work as scratch.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA.
+ */
+int flide_fork_attn(const void *q, const void *k, const void *v,
+                    const void *past_k, const void *past_v, int32_t past_rows,
+                    flide_tree_index *idx, int32_t Hq, int32_t Hkv, int32_t d,
+                    int32_t dtype, float scale, void *out, int32_t flags,
+                    flide_stream stream);
+
+/*
+ * Gated DeltaNet fork scan (kongchang.com, Gated DeltaNet box: each
+ * branch evolves its own recurrent state in isolation order; techfi24.com:
+ * the state is cloned at the decision point, not recomputed).  Per head, with
+ * state S (dv x dk, fp32) and alpha = exp(g):
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t.
+ * The root of request r starts from state_in[r] (zeros if state_in is NULL);
+ * every other node starts from its parent's end state.  The end state of every
+ * node with a slot (roots and inner nodes) is written to
+ * node_state[idx->state_slot[n]]; the root's is the request's checkpoint.
+ *   q, k [T, H, dk] dtype;  v [T, H, dv] dtype;  g, beta [T, H] fp32
+ *   state_in [R, H, dv, dk] fp32 or NULL
+ *   out [T, H, dv] dtype
+ *   node_state [n_state_slots, H, dv, dk] fp32 (required)
+ * Device error FLIDE_ERR_CAPACITY if the tree needs more than n_state_slots.
+ * Supported: dk in {32, 64, 128, 256}, dv a multiple of 32.
+ */
+int flide_fork_gdn(const void *q, const void *k, const void *v,
+                   const float *g, const float *beta, const float *state_in,
+                   flide_tree_index *idx, int32_t H, int32_t dk, int32_t dv,
+                   int32_t dtype, void *out, float *node_state,
+                   int32_t n_state_slots, int32_t flags, flide_stream stream);
+
+/*
+ * Checkpoint save (kongchang.com, "ForkAttention": growing agent histories
+ * resume from checkpoints saved in earlier passes).  For every request r the
+ * shared prefix becomes history: rows [ckpt_start[r], ckpt_start[r+1]) of
+ * ckpt_k/ckpt_v receive the request's past rows followed by its root rows, and
+ * ckpt_S[r] receives the root's end state node_state[state_slot[root]] (zeros
+ * for a request without nodes).  A later batch passes ckpt_k/ckpt_v as its
+ * past_k/past_v and past_len[r] = ckpt_start[r+1] - ckpt_start[r].
+ *   k, v   [T, Hkv, d] dtype         past_k, past_v as in flide_fork_attn
+ *   node_state as written by flide_fork_gdn (may be NULL with H == 0)
+ *   ckpt_k, ckpt_v [ckpt_rows, Hkv, d] dtype;  ckpt_S [R, H, dv, dk] fp32
+ * Device error FLIDE_ERR_CAPACITY if the checkpoint needs more than ckpt_rows.
+ */
+int flide_state_save(const flide_tree_index *idx, const void *k, const void *v,
+                     const void *past_k, const void *past_v, int32_t Hkv,
+                     int32_t d, int32_t dtype, const float *node_state,
+                     int32_t H, int32_t dk, int32_t dv, void *ckpt_k,
+                     void *ckpt_v, float *ckpt_S, int32_t ckpt_rows,
+                     flide_stream stream);
+
+/*
+ * Checkpoint resume: gathers saved checkpoints into the past inputs of a
+ * new batch.  Request r of the new batch resumes checkpoint src_req[r] of a
+ * saved set (src_req[r] < 0: a fresh request with no past).  Writes
+ * past_len[r] (int32, the new tree's past lengths), the packed
+ * past_k/past_v rows (request order) and state_in[r] (zeros when fresh).
+ *   src_ckpt_start [src_R+1] int32 (the saved index's ckpt_start)
+ *   src_k, src_v [*, Hkv, d] dtype; src_S [src_R, H, dv, dk] fp32
+ *   src_req [R] int32 (device)
+ *   past_k, past_v [past_rows, Hkv, d]; state_in [R, H, dv, dk] fp32
+ * Writes FLIDE_ERR_CAPACITY / FLIDE_ERR_INVALID to *status (device int32) if
+ * the rows exceed past_rows or src_req is out of range.
+ */
+int flide_state_resume(int32_t R, const int32_t *src_req, int32_t src_R,
+                       const int32_t *src_ckpt_start, const void *src_k,
+                       const void *src_v, const float *src_S, int32_t Hkv,
+                       int32_t d, int32_t dtype, int32_t H, int32_t dk,
+                       int32_t dv, int32_t *past_len, void *past_k,
+                       void *past_v, int32_t past_rows, float *state_in,
+                       int32_t *status, flide_stream stream);
+
+/* Static message for a status code. */
+const char *flide_strerror(int32_t code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLIDE_H */

@@ -1,0 +1,228 @@
+"""Thin Python binding over libflide.so (include/flide.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  The
+binding raises if the library is missing -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libflide.so")
+
+OK, ERR_INVALID, ERR_SHAPE, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT = range(6)
+F32, BF16 = 0, 1
+FLAG_PORTABLE = 1
+COUNTS = 16
+CNT = dict(N=0, T=1, PAST=2, DEPTH=3, SLOTS=4, BRANCH_TOK=5, ROOT_TOK=6, CKPT_ROWS=7)
+
+# names and order of the int32* members of flide_tree_index
+INDEX_ARRAYS = ["status", "counts", "node_start", "node_req", "depth", "anc_ptr", "anc_node",
+                "ctx_len", "token_node", "token_pos", "past_start", "req_node", "level_ptr",
+                "level_node", "state_slot", "ckpt_start", "work"]
+
+# every extern "C" symbol declared in include/flide.h
+SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build",
+           "flide_fork_attn", "flide_fork_gdn", "flide_state_save", "flide_state_resume",
+           "flide_strerror"]
+
+
+class FlideError(RuntimeError):
+    def __init__(self, code, where=""):
+        msg = _lib().flide_strerror(code).decode() if _LIB is not None else str(code)
+        super().__init__(f"{where}: flide status {code} ({msg})")
+        self.code = code
+
+
+class TreeDesc(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_int32), ("N", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("max_depth", ctypes.c_int32), ("req_node_ptr", ctypes.c_void_p),
+                ("parent", ctypes.c_void_p), ("seg_len", ctypes.c_void_p),
+                ("past_len", ctypes.c_void_p)]
+
+
+class TreeIndexC(ctypes.Structure):
+    _fields_ = ([("R", ctypes.c_int32), ("N", ctypes.c_int32), ("T", ctypes.c_int32),
+                 ("max_depth", ctypes.c_int32)]
+                + [(n, ctypes.c_void_p) for n in INDEX_ARRAYS]
+                + [("work_len", ctypes.c_int64)])
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m tree_forked_decision_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        lib.flide_tree_index_bytes.argtypes = [I32, I32, I32, I32]
+        lib.flide_tree_index_bytes.restype = ctypes.c_size_t
+        lib.flide_tree_index_init.argtypes = [P, P, ctypes.c_size_t, I32, I32, I32, I32]
+        lib.flide_tree_index_init.restype = ctypes.c_int
+        lib.flide_tree_build.argtypes = [P, P, P]
+        lib.flide_tree_build.restype = ctypes.c_int
+        lib.flide_fork_attn.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32, F, P, I32, P]
+        lib.flide_fork_attn.restype = ctypes.c_int
+        lib.flide_fork_gdn.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, P, P, I32, I32, P]
+        lib.flide_fork_gdn.restype = ctypes.c_int
+        lib.flide_state_save.argtypes = [P, P, P, P, P, I32, I32, I32, P, I32, I32, I32, P, P, P,
+                                         I32, P]
+        lib.flide_state_save.restype = ctypes.c_int
+        lib.flide_state_resume.argtypes = [I32, P, I32, P, P, P, P, I32, I32, I32, I32, I32, I32,
+                                           P, P, P, I32, P, P, P]
+        lib.flide_state_resume.restype = ctypes.c_int
+        lib.flide_strerror.argtypes = [ctypes.c_int32]
+        lib.flide_strerror.restype = ctypes.c_char_p
+        _LIB = lib
+    return _LIB
+
+
+def load():
+    """Loads libflide.so (raises if absent) and returns the ctypes handle."""
+    return _lib()
+
+
+def _check(code, where):
+    if code != OK:
+        raise FlideError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+class TreeIndex:
+    """Device-resident tree index over one torch-allocated buffer."""
+
+    def __init__(self, R: int, N: int, T: int, max_depth: int, device="cuda"):
+        lib = _lib()
+        nbytes = lib.flide_tree_index_bytes(R, N, T, max_depth)
+        if nbytes == 0:
+            raise FlideError(ERR_SHAPE, "flide_tree_index_bytes")
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.c = TreeIndexC()
+        _check(lib.flide_tree_index_init(ctypes.byref(self.c), ctypes.c_void_p(self.buf.data_ptr()),
+                                         nbytes, R, N, T, max_depth), "flide_tree_index_init")
+        self.R, self.N, self.T, self.max_depth = R, N, T, max_depth
+
+    def array(self, name: str, n: int) -> torch.Tensor:
+        """int32 view of one index array (first n entries)."""
+        off = getattr(self.c, name) - self.buf.data_ptr()
+        return self.buf[off:off + 4 * n].view(torch.int32)
+
+    def status(self) -> int:
+        return int(self.array("status", 1).item())
+
+    def counts(self) -> dict:
+        c = self.array("counts", COUNTS).cpu().tolist()
+        return {k: c[v] for k, v in CNT.items()}
+
+
+class DeviceTree:
+    """Device copies of a tree's arrays (the flide_tree_desc inputs)."""
+
+    def __init__(self, req_node_ptr, parent, seg_len, past_len, max_depth: int,
+                 N: int | None = None, T: int | None = None, device="cuda"):
+        as_i32 = lambda a: torch.as_tensor(np.asarray(a, np.int32)).to(device)
+        self.req_node_ptr = as_i32(req_node_ptr)
+        self.parent = as_i32(parent)
+        self.seg_len = as_i32(seg_len)
+        self.past_len = as_i32(past_len)
+        self.R = len(req_node_ptr) - 1
+        self.N = int(N if N is not None else max(len(parent), 1))
+        self.T = int(T if T is not None else max(int(np.sum(seg_len)), 1))
+        self.max_depth = int(max_depth)
+        if len(parent) == 0:  # keep valid pointers for empty batches
+            self.parent = torch.full((1,), -1, dtype=torch.int32, device=device)
+            self.seg_len = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def desc(self) -> TreeDesc:
+        return TreeDesc(self.R, self.N, self.T, self.max_depth, self.req_node_ptr.data_ptr(),
+                        self.parent.data_ptr(), self.seg_len.data_ptr(), self.past_len.data_ptr())
+
+
+def tree_build(tree: DeviceTree, index: TreeIndex, stream=None):
+    d = tree.desc()
+    _check(_lib().flide_tree_build(ctypes.byref(d), ctypes.byref(index.c), _stream(stream)),
+           "flide_tree_build")
+
+
+def fork_attn(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None, out=None,
+              flags: int = 0, stream=None):
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    past_rows = 0 if past_k is None else past_k.shape[0]
+    if past_rows == 0:
+        past_k = past_v = None
+    _check(_lib().flide_fork_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(past_k), _ptr(past_v),
+                                  past_rows, ctypes.byref(index.c), Hq, Hkv, d, _dtype_code(q),
+                                  float(scale), _ptr(out), flags, _stream(stream)),
+           "flide_fork_attn")
+    return out
+
+
+def fork_gdn(q, k, v, g, beta, index: TreeIndex, node_state, state_in=None, out=None,
+             flags: int = 0, stream=None):
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    _check(_lib().flide_fork_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+                                 ctypes.byref(index.c), H, dk, dv, _dtype_code(q), _ptr(out),
+                                 _ptr(node_state), node_state.shape[0], flags, _stream(stream)),
+           "flide_fork_gdn")
+    return out
+
+
+def state_save(index: TreeIndex, k, v, ckpt_k, ckpt_v, ckpt_S, past_k=None, past_v=None,
+               node_state=None, stream=None):
+    Hkv, d = (k.shape[1], k.shape[2]) if k is not None else (0, 0)
+    H = dv = dk = 0
+    if node_state is not None:
+        _, H, dv, dk = node_state.shape
+    dt = _dtype_code(k) if k is not None else BF16
+    _check(_lib().flide_state_save(ctypes.byref(index.c), _ptr(k), _ptr(v), _ptr(past_k),
+                                   _ptr(past_v), Hkv, d, dt, _ptr(node_state), H, dk, dv,
+                                   _ptr(ckpt_k), _ptr(ckpt_v), _ptr(ckpt_S),
+                                   0 if ckpt_k is None else ckpt_k.shape[0], _stream(stream)),
+           "flide_state_save")
+
+
+def state_resume(src_req, src_ckpt_start, src_k, src_v, src_S, past_len, past_k, past_v,
+                 state_in, status, stream=None):
+    R = src_req.shape[0]
+    src_R = src_ckpt_start.shape[0] - 1
+    Hkv, d = src_k.shape[1], src_k.shape[2]
+    H = dv = dk = 0
+    if state_in is not None:
+        _, H, dv, dk = state_in.shape
+    _check(_lib().flide_state_resume(R, _ptr(src_req), src_R, _ptr(src_ckpt_start), _ptr(src_k),
+                                     _ptr(src_v), _ptr(src_S), Hkv, d, _dtype_code(src_k), H, dk,
+                                     dv, _ptr(past_len), _ptr(past_k), _ptr(past_v),
+                                     past_k.shape[0], _ptr(state_in), _ptr(status),
+                                     _stream(stream)),
+           "flide_state_resume")
