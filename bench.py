@@ -1,0 +1,539 @@
+#!/usr/bin/env python
+"""Throughput of the ForkAttention hot path: branch-token evals/s.
+
+One step = one pass of the whole path over one batch of synthetic decision
+requests already resident in HBM: tree-index build -> fork attention ->
+Gated DeltaNet fork scan -> checkpoint save, all through libflide.so's C ABI
+on one stream.  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on the same workload
+
+Multi-GPU (torchrun): requests are independent, so every rank runs its own
+batch (seed offset by rank) with no data-path collective -- weak scaling; the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tree_forked_decision_b200 import flide, inputs  # noqa: E402
+
+METRIC = "branch-token evals/sec (fork attn + GDN layer, 1 B200); % of roofline"
+UNIT = "branch-token evals/s"
+DEFAULT_WORKLOAD = "large_fanout_bf16"
+# fallbacks when the measured-peaks file is absent (earlier measurements on this machine)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic (measurement only)
+# ---------------------------------------------------------------------------
+
+def isolated_positions(tree: inputs.Tree) -> np.ndarray:
+    """Length of each token's isolated sequence before it (past + ancestors +
+    earlier tokens of its node), from the tree structure."""
+    rp, pa, sl, pl = tree.arrays()
+    before = np.zeros(tree.N, np.int64)
+    for r in range(tree.R):
+        for n in range(rp[r], rp[r + 1]):
+            before[n] = pl[r] if pa[n] < 0 else before[rp[r] + pa[n]] + sl[rp[r] + pa[n]]
+    offs = np.concatenate([np.arange(s) for s in sl]) if tree.N else np.zeros(0, np.int64)
+    return np.repeat(before, sl) + offs
+
+
+def attn_work(tree, a):
+    """Algorithmic FLOPs (QK^T + PV over exactly the visible keys) and bytes
+    (q, k, v, out once, plus the past rows once) of one fork-attention launch."""
+    d, Hq, Hkv = a["d"], a["Hq"], a["Hkv"]
+    vis = isolated_positions(tree) + 1
+    flops = 4.0 * d * Hq * float(vis.sum())
+    es = 2 if a["q"].dtype == torch.bfloat16 else 4
+    byts = es * d * (2 * tree.T * Hq + 2 * tree.T * Hkv + 2 * tree.P_past * Hkv)
+    return flops, byts
+
+
+def gdn_work(tree, g, slots):
+    """Algorithmic bytes of one GDN fork scan: q, k, v, out, g, beta once, plus
+    one fp32 state write per saved node and one read per child / resumed root."""
+    H, dk, dv = g["H"], g["dk"], g["dv"]
+    es = 2 if g["q"].dtype == torch.bfloat16 else 4
+    state = 4 * H * dk * dv
+    reads = int(tree.N - tree.R) + int(np.sum(tree.past_len > 0))
+    byts = tree.T * H * ((2 * dk + 2 * dv) * es + 8) + state * (slots + reads)
+    return byts
+
+
+# ---------------------------------------------------------------------------
+# device step
+# ---------------------------------------------------------------------------
+
+class Step:
+    """Device buffers and one call sequence of the hot path."""
+
+    def __init__(self, tree, a, g, device):
+        self.tree, self.a, self.g = tree, a, g
+        self.dt = flide.DeviceTree(*tree.arrays(), max_depth=max(tree.levels, 1), device=device)
+        self.idx = flide.TreeIndex(self.dt.R, self.dt.N, self.dt.T, self.dt.max_depth, device=device)
+        dev = lambda t: t.to(device, non_blocking=False).contiguous()
+        self.launches = 2
+        if a is not None:
+            self._init_attn(tree, a, dev, device)
+        if g is not None:
+            self._init_gdn(tree, g, dev, device)
+
+    def _init_attn(self, tree, a, dev, device):
+        self.q, self.k, self.v = dev(a["q"]), dev(a["k"]), dev(a["v"])
+        self.pk = dev(a["past_k"]) if a["past_k"].shape[0] else None
+        self.pv = dev(a["past_v"]) if a["past_v"].shape[0] else None
+        self.o = torch.empty_like(self.q)
+        self.scale = 1.0 / math.sqrt(a["d"])
+        self.launches += 2
+        self.ckpt_rows = tree.P_past + tree.root_tokens
+        self.ck = torch.empty((max(self.ckpt_rows, 1), a["Hkv"], a["d"]), dtype=self.k.dtype,
+                              device=device)
+        self.cv = torch.empty_like(self.ck)
+        self.launches += 1
+
+    def _init_gdn(self, tree, g, dev, device):
+        self.gq, self.gk, self.gv = dev(g["q"]), dev(g["k"]), dev(g["v"])
+        self.gg, self.gb = dev(g["g"]), dev(g["beta"])
+        self.state_in = dev(g["state_in"]) if np.any(tree.past_len > 0) else None
+        self.go = torch.empty((tree.T, g["H"], g["dv"]), dtype=self.gq.dtype, device=device)
+        # node-state capacity: roots + every node that has children
+        has_child = np.zeros(tree.N, bool)
+        rp = tree.req_node_ptr
+        for r in range(tree.R):
+            for n in range(rp[r] + 1, rp[r + 1]):
+                has_child[rp[r] + tree.parent[n]] = True
+        roots = rp[:-1][rp[:-1] < rp[1:]]
+        has_child[roots] = True
+        self.slots = max(int(has_child.sum()), 1)
+        self.node_state = torch.empty((self.slots, g["H"], g["dv"], g["dk"]), dtype=torch.float32,
+                                      device=device)
+        self.cS = torch.empty((tree.R, g["H"], g["dv"], g["dk"]), dtype=torch.float32, device=device)
+        self.launches += (self.dt.max_depth + 1) + 1
+
+    def run(self, ev=None):
+        """tree build -> fork attention -> GDN fork scan -> checkpoint save;
+        ev = 3 CUDA events recorded around the two layers."""
+        a, g = self.a is not None, self.g is not None
+        flide.tree_build(self.dt, self.idx)
+        if ev is not None:
+            ev[0].record()
+        if a:
+            flide.fork_attn(self.q, self.k, self.v, self.idx, self.scale, past_k=self.pk,
+                            past_v=self.pv, out=self.o)
+        if ev is not None:
+            ev[1].record()
+        if g:
+            flide.fork_gdn(self.gq, self.gk, self.gv, self.gg, self.gb, self.idx,
+                           self.node_state, state_in=self.state_in, out=self.go)
+        if ev is not None:
+            ev[2].record()
+        flide.state_save(self.idx, self.k if a else None, self.v if a else None,
+                         self.ck if a else None, self.cv if a else None,
+                         self.cS if g else None, past_k=self.pk if a else None,
+                         past_v=self.pv if a else None,
+                         node_state=self.node_state if g else None)
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_rate(tree, a, g, attn_rows: int, gdn_pairs: int, seed: int = 0):
+    """Times the oracle on a seeded uniform sample of the workload's units --
+    attention query rows and GDN (request, head) pairs -- and scales each time
+    by (all units / sampled units).  Returns (evals/s, description, threads)."""
+    import oracle  # test infrastructure: only this leg and the reference arm use it
+
+    rng = np.random.default_rng(seed)
+    f32 = lambda t: t.float().numpy()
+    T, Hq = tree.T, a["Hq"]
+    n_rows = T * Hq
+    pick = rng.choice(n_rows, size=min(attn_rows, n_rows), replace=False)
+    rows = np.stack([pick // Hq, pick % Hq], 1).astype(np.int32)
+    qa, ka, va, pka, pva = f32(a["q"]), f32(a["k"]), f32(a["v"]), f32(a["past_k"]), f32(a["past_v"])
+    t0 = time.perf_counter()
+    oracle.attention_rows(tree.arrays(), qa, ka, va, pka, pva, 1.0 / math.sqrt(a["d"]), rows)
+    t_attn = (time.perf_counter() - t0) * n_rows / len(rows)
+    del qa, ka, va
+    H = g["H"]
+    all_pairs = [(r, h) for r in range(tree.R) for h in range(H)]
+    sel = rng.choice(len(all_pairs), size=min(gdn_pairs, len(all_pairs)), replace=False)
+    heads = sorted({all_pairs[i][1] for i in sel})
+    # slice the selected heads so the oracle reads only their data
+    hq = lambda t: np.ascontiguousarray(f32(t)[:, heads])
+    pairs = [(all_pairs[i][0], heads.index(all_pairs[i][1])) for i in sel]
+    st = f32(g["state_in"])[:, heads] if np.any(tree.past_len > 0) else None
+    gq, gk, gv, gg, gb = hq(g["q"]), hq(g["k"]), hq(g["v"]), hq(g["g"]), hq(g["beta"])
+    t0 = time.perf_counter()
+    oracle.gdn(tree.arrays(), gq, gk, gv, gg, gb, state_in=st, memoise=True, pairs=pairs)
+    t_gdn = (time.perf_counter() - t0) * len(all_pairs) / len(sel)
+    rate = tree.branch_tokens / (t_attn + t_gdn)
+    desc = (f"{len(rows)} of {n_rows} attention query rows and {len(sel)} of {len(all_pairs)} "
+            f"GDN (request, head) pairs (memoised oracle), seeded uniform sample; each time "
+            f"scaled by all/sampled units: attention {t_attn:.1f} s + GDN {t_gdn:.1f} s "
+            f"per step extrapolated")
+    return rate, desc, oracle.num_threads()
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            pk = json.load(fh)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_for(kernel_name: str, src_file: str):
+    """dram read+write bytes per launch for `kernel_name` from the committed ncu
+    summary, or None when the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel_name]
+    except (OSError, ValueError, KeyError):
+        return None
+    src = os.path.join(ROOT, "tree_forked_decision_b200", "csrc", src_file)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if rec.get("source_sha") != sha:
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    tree, a, g, dtype = inputs.make_inputs(args.workload, seed=args.seed)
+    for _ in range(args.warmup):
+        cpu_oracle_rate(tree, a, g, args.ref_rows, args.ref_pairs, seed=1)
+    rates, desc, threads = [], "", 1
+    t_start = time.perf_counter()
+    for s in range(args.steps):
+        r, desc, threads = cpu_oracle_rate(tree, a, g, args.ref_rows, args.ref_pairs, seed=2 + s)
+        rates.append(r)
+    wall = time.perf_counter() - t_start
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * tree.branch_tokens / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "requests": tree.R, "tokens": tree.T,
+                   "branch_tokens": tree.branch_tokens, "seed": args.seed,
+                   "oracle": "plain C fp64 oracle (memoised GDN), OpenMP over units"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="flide", choices=["flide", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=None)
+    ap.add_argument("--layers", default="both", choices=["both", "attn", "gdn"],
+                    help="profiling aid: run one layer only (not a headline number)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=6000)
+    ap.add_argument("--cpu-pairs", type=int, default=16)
+    ap.add_argument("--ref-rows", type=int, default=2000)
+    ap.add_argument("--ref-pairs", type=int, default=16)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    ws, rank, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    pg = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+        pg = dist
+    flide.load()
+
+    spec = inputs.WORKLOADS[args.workload]
+    seed = (args.seed if args.seed is not None else spec["idx"]) + 1000 * rank
+    tree, a, g, dtype = inputs.make_inputs(args.workload, seed=seed)
+    if args.layers == "attn":
+        g = None
+    elif args.layers == "gdn":
+        a = None
+    if a is None and g is None:
+        raise SystemExit(f"{args.workload}: no layer left to run")
+    if args.layers == "both" and (a is None or g is None):
+        raise SystemExit(f"{args.workload} lacks one of the two layers; use --layers")
+    step = Step(tree, a, g, device)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up, then check the path ran clean
+    for _ in range(max(args.warmup, 0)):
+        step.run()
+    torch.cuda.synchronize()
+    if step.idx.status() != 0:
+        raise SystemExit(f"device status {step.idx.status()} after warm-up")
+
+    # timed region: inputs resident in HBM (GBs per step, far above the 126 MB L2)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        start.record()
+        for i in range(args.steps):
+            step.run(evs[i])
+        stop.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = start.elapsed_time(stop)
+    attn_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    gdn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if step.idx.status() != 0:
+        raise SystemExit(f"device status {step.idx.status()} in the timed region")
+    if pg is not None:
+        t = torch.tensor([ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    units = tree.branch_tokens * args.steps * ws
+    value = units / (ms / 1000.0)
+
+    # end to end through the public API with host buffers: H2D of every input
+    # from pinned memory, the call sequence, D2H of every branch token's output
+    e2e = None
+    if not args.no_e2e and a is not None and g is not None:
+        host = {}
+        for pre, src, names in (("a_", a, ("q", "k", "v", "past_k", "past_v")),
+                                ("g_", g, ("q", "k", "v", "g", "beta", "state_in"))):
+            for nm in names:
+                t = src[nm]
+                host[pre + nm] = t.pin_memory() if t.numel() else None
+        if step.state_in is None:
+            host["g_state_in"] = None
+        tree_host = [torch.from_numpy(np.ascontiguousarray(x)).pin_memory() for x in tree.arrays()]
+        # branch tokens are not contiguous across requests: gather their rows
+        rp = tree.req_node_ptr
+        starts = np.concatenate([[0], np.cumsum(tree.seg_len)])
+        br_rows = np.concatenate([np.arange(starts[rp[r] + 1], starts[rp[r + 1]])
+                                  for r in range(tree.R) if rp[r + 1] > rp[r]]).astype(np.int64)
+        br_idx = torch.from_numpy(br_rows).to(device)
+        out_a = torch.empty((len(br_rows),) + tuple(step.o.shape[1:]), dtype=step.o.dtype).pin_memory()
+        out_g = torch.empty((len(br_rows),) + tuple(step.go.shape[1:]), dtype=step.go.dtype).pin_memory()
+        status_h = torch.empty(1, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        h2d += sum(t.numel() * t.element_size() for t in tree_host)
+        d2h = out_a.numel() * out_a.element_size() + out_g.numel() * out_g.element_size() + 4
+
+        def e2e_step():
+            for dst, src in ((step.dt.req_node_ptr, tree_host[0]), (step.dt.parent, tree_host[1]),
+                             (step.dt.seg_len, tree_host[2]), (step.dt.past_len, tree_host[3])):
+                dst.copy_(src, non_blocking=True)
+            step.q.copy_(host["a_q"], non_blocking=True)
+            step.k.copy_(host["a_k"], non_blocking=True)
+            step.v.copy_(host["a_v"], non_blocking=True)
+            if step.pk is not None:
+                step.pk.copy_(host["a_past_k"], non_blocking=True)
+                step.pv.copy_(host["a_past_v"], non_blocking=True)
+            step.gq.copy_(host["g_q"], non_blocking=True)
+            step.gk.copy_(host["g_k"], non_blocking=True)
+            step.gv.copy_(host["g_v"], non_blocking=True)
+            step.gg.copy_(host["g_g"], non_blocking=True)
+            step.gb.copy_(host["g_beta"], non_blocking=True)
+            if step.state_in is not None:
+                step.state_in.copy_(host["g_state_in"], non_blocking=True)
+            step.run()
+            out_a.copy_(step.o.index_select(0, br_idx), non_blocking=True)
+            out_g.copy_(step.go.index_select(0, br_idx), non_blocking=True)
+            status_h.copy_(step.idx.array("status", 1), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if pg is not None:
+            t = torch.tensor([ems], device=device)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ems = float(t.item())
+        if int(status_h.item()) != 0:
+            raise SystemExit(f"device status {int(status_h.item())} in the e2e leg")
+        e2e = {"value": tree.branch_tokens * n_e2e * ws / (ems / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e, "ms_per_step": ems / n_e2e}
+
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    kernels, roofline = {}, None
+    if g is not None:
+        gbytes = gdn_work(tree, g, step.slots)
+        gdn_gbs = gbytes / (gdn_ms / 1000.0) / 1e9
+        kernels["fork_gdn"] = {"ms": gdn_ms, "algorithmic_bytes": gbytes, "gbs": gdn_gbs,
+                               "frac_of_hbm_peak": gdn_gbs / hbm, "bound": "hbm"}
+        roofline = {
+            "kernel": "gdn_level_kernel (GDN fork scan)", "bound": "hbm", "achieved": gdn_gbs,
+            "peak": hbm, "unit": "GB/s", "frac": gdn_gbs / hbm,
+            "traffic": traffic_for("gdn_level_kernel", "gdn_portable.cu"),
+            "peak_source": f"{peak_src}: HBM copy bandwidth",
+            "algorithmic_bytes_per_launch": gbytes, "avg_launch_ms": gdn_ms}
+    if a is not None:
+        flops, abytes = attn_work(tree, a)
+        achieved = flops / (attn_ms / 1000.0) / 1e12
+        kernels["fork_attn"] = {"ms": attn_ms, "tflops": achieved,
+                                "frac_of_tensor_peak": achieved / peak, "bound": "tensor"}
+        # the dominant kernel of the step
+        if g is None or attn_ms >= gdn_ms:
+            roofline = {
+                "kernel": "attn_tc_kernel (fork attention, tcgen05)",
+                "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic_for("attn_tc_kernel", "attn_tc.cu"),
+                "peak_source": f"{peak_src}: sustained dense bf16 (kernel timed inside a long step)",
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
+                "avg_launch_ms": attn_ms,
+            }
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and a is not None and g is not None:
+        rate, desc, threads = cpu_oracle_rate(tree, a, g, args.cpu_rows, args.cpu_pairs)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "requests_per_gpu": tree.R, "tokens_per_gpu": tree.T,
+                   "branch_tokens_per_gpu": tree.branch_tokens,
+                   "attn": f"Hq={a['Hq']} Hkv={a['Hkv']} d={a['d']}" if a is not None else None,
+                   "gdn": f"H={g['H']} dk={g['dk']} dv={g['dv']}" if g is not None else None,
+                   "layers": args.layers,
+                   "l2": "inputs larger than L2 (GBs per step), no flush",
+                   "parallelism": f"dp{ws} (independent requests per rank)", "seed": seed},
+        "roofline": roofline,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": step.launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -18,8 +18,10 @@ parent[i] < i; node 0 of every request is its root.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
 import numpy as np
 import torch
@@ -148,6 +150,31 @@ def random_tree(rng: np.random.Generator, R: int, max_nodes: int = 8,
     return _tree(reqs, levels)
 
 
+_CHUNK = 1 << 24  # elements per independently seeded block of normals
+
+
+def normals(rng: np.random.Generator, shape) -> np.ndarray:
+    """float32 N(0,1) array of `shape`.  Large arrays are filled in blocks of
+    2^24 elements, each from its own generator seeded by `rng`, on several
+    threads; the values depend only on rng's state and the shape."""
+    n = int(np.prod(shape))
+    out = np.empty(n, np.float32)
+    blocks = (n + _CHUNK - 1) // _CHUNK
+    seeds = rng.integers(0, 2**63 - 1, size=max(blocks, 1))
+
+    def fill(b):
+        sl = slice(b * _CHUNK, min(n, (b + 1) * _CHUNK))
+        np.random.default_rng(int(seeds[b])).standard_normal(out=out[sl], dtype=np.float32)
+
+    if blocks <= 1:
+        if n:
+            fill(0)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(blocks)))
+    return out.reshape(shape)
+
+
 def _to(x: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(x)).to(dtype)
 
@@ -156,18 +183,19 @@ def attn_inputs(tree: Tree, Hq: int, Hkv: int, d: int, dtype: torch.dtype,
                 rng: np.random.Generator):
     """q [T,Hq,d], k,v [T,Hkv,d], past_k,past_v [sum(past),Hkv,d]; N(0,1)."""
     T, P = tree.T, tree.P_past
-    q = rng.standard_normal((T, Hq, d), dtype=np.float32)
-    k = rng.standard_normal((T, Hkv, d), dtype=np.float32)
-    v = rng.standard_normal((T, Hkv, d), dtype=np.float32)
-    pk = rng.standard_normal((P, Hkv, d), dtype=np.float32)
-    pv = rng.standard_normal((P, Hkv, d), dtype=np.float32)
+    q = normals(rng, (T, Hq, d))
+    k = normals(rng, (T, Hkv, d))
+    v = normals(rng, (T, Hkv, d))
+    pk = normals(rng, (P, Hkv, d))
+    pv = normals(rng, (P, Hkv, d))
     return dict(q=_to(q, dtype), k=_to(k, dtype), v=_to(v, dtype),
                 past_k=_to(pk, dtype), past_v=_to(pv, dtype))
 
 
-def _l2n(x: np.ndarray) -> np.ndarray:
-    n = np.sqrt((x.astype(np.float32) ** 2).sum(-1, keepdims=True, dtype=np.float32))
-    return (x / np.maximum(n, np.float32(1e-6))).astype(np.float32)
+def _l2n(x: np.ndarray) -> torch.Tensor:
+    """Rows scaled to unit L2 norm, in float32."""
+    t = torch.from_numpy(x)
+    return t / torch.linalg.vector_norm(t, dim=-1, keepdim=True).clamp_min(1e-6)
 
 
 def gdn_inputs(tree: Tree, H: int, dk: int, dv: int, dtype: torch.dtype,
@@ -178,9 +206,9 @@ def gdn_inputs(tree: Tree, H: int, dk: int, dv: int, dtype: torch.dtype,
     [R,H,dv,dk] float32: N(0, state_scale^2) for requests with past history,
     zero otherwise."""
     T, R = tree.T, tree.R
-    q = _l2n(rng.standard_normal((T, H, dk), dtype=np.float32))
-    k = _l2n(rng.standard_normal((T, H, dk), dtype=np.float32))
-    v = rng.standard_normal((T, H, dv), dtype=np.float32)
+    q = _l2n(normals(rng, (T, H, dk)))
+    k = _l2n(normals(rng, (T, H, dk)))
+    v = normals(rng, (T, H, dv))
     x = rng.standard_normal((T, H)).astype(np.float64)
     g = (-gate_scale * np.logaddexp(0.0, x)).astype(np.float32)
     y = rng.standard_normal((T, H)).astype(np.float64)
@@ -188,8 +216,8 @@ def gdn_inputs(tree: Tree, H: int, dk: int, dv: int, dtype: torch.dtype,
     state = np.zeros((R, H, dv, dk), np.float32)
     for r in range(R):
         if tree.past_len[r] > 0:
-            state[r] = rng.standard_normal((H, dv, dk), dtype=np.float32) * np.float32(state_scale)
-    return dict(q=_to(q, dtype), k=_to(k, dtype), v=_to(v, dtype),
+            state[r] = normals(rng, (H, dv, dk)) * np.float32(state_scale)
+    return dict(q=q.to(dtype), k=k.to(dtype), v=_to(v, dtype),
                 g=torch.from_numpy(g), beta=torch.from_numpy(beta),
                 state_in=torch.from_numpy(state))
 
