@@ -170,6 +170,38 @@ int flide_fork_attn(const void *q, const void *k, const void *v,
                     flide_stream stream);
 
 /*
+ * Fork attention without caller-provided scratch.  (No counterpart in the
+ * pages: this is a library convenience, not part of the method.)
+ *
+ * flide_fork_attn keeps a small per-call work table in idx->work, so whoever
+ * lays out the index must also reserve that scratch and let every attention
+ * call write into it.  Some callers cannot: the index may have been built by
+ * another component into a fixed region they may only read, or the caller may
+ * run inside a framework whose device memory pool is closed to new
+ * allocations, so it can neither grow the index nor allocate a scratch buffer
+ * of its own.  This entry point computes exactly what flide_fork_attn computes
+ * (same arguments, same kernels) but never touches idx->work and allocates
+ * nothing: the work table lives in a fixed 64 KB array compiled into
+ * libflide.so, present on every GPU that loads the library until the process
+ * exits.
+ *   - At most 16384 requests (idx->R); larger indices return
+ *     FLIDE_ERR_CAPACITY before any work is queued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture that should contain it.
+ *   - All calls on a device share the one array.  Each call writes every entry
+ *     it reads before reading it, so nothing needs clearing between calls, but
+ *     calls whose executions overlap on the GPU (for example on two streams)
+ *     race on it: order them on one stream or with events.
+ *   - Returns as flide_fork_attn; device-detected errors go to idx->status.
+ */
+int flide_fork_attn_noalloc(const void *q, const void *k, const void *v,
+                            const void *past_k, const void *past_v, int32_t past_rows,
+                            const flide_tree_index *idx, int32_t Hq, int32_t Hkv,
+                            int32_t d, int32_t dtype, float scale, void *out,
+                            int32_t flags, flide_stream stream);
+
+/*
  * Gated DeltaNet fork scan (kongchang.com, Gated DeltaNet box: each
  * branch evolves its own recurrent state in isolation order; techfi24.com:
  * the state is cloned at the decision point, not recomputed).  Per head, with

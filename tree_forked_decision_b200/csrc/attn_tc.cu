@@ -42,6 +42,9 @@
 #include "sm100.cuh"
 
 namespace flide {
+int fork_attn_portable(const void *q, const void *k, const void *v, const void *pk,
+                       const void *pv, const flide_tree_index *x, int Hq, int Hkv, int d,
+                       int dtype, float scale, void *out, cudaStream_t s);
 namespace {
 
 using namespace sm100;
@@ -569,3 +572,59 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
 }
 
 }  // namespace flide
+
+// ---- entry point without caller-provided scratch ---------------------------
+//
+// flide_fork_attn keeps its per-call work table (one int32 per request plus
+// one) in the caller's index buffer, idx->work.  flide_fork_attn_noalloc runs
+// the same kernels but takes that table from the fixed array below, which
+// every GPU that loads libflide.so holds until the process exits (64 KB).
+
+namespace flide {
+namespace {
+
+constexpr int kNoAllocMaxRequests = 16384;
+static __device__ __align__(256) int32_t g_noalloc_work[kNoAllocMaxRequests + 1];
+
+// Device address of g_noalloc_work on the current device.  In host code the
+// array's name only stands in for the symbol, so the address is looked up once
+// per device with that device current and cached.
+int32_t *noalloc_work_ptr() {
+  static int32_t *cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_work) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64) cached[dev] = (int32_t *)p;
+  return (int32_t *)p;
+}
+
+}  // namespace
+}  // namespace flide
+
+extern "C" int flide_fork_attn_noalloc(const void *q, const void *k, const void *v,
+                                       const void *past_k, const void *past_v,
+                                       int32_t past_rows, const flide_tree_index *idx,
+                                       int32_t Hq, int32_t Hkv, int32_t d, int32_t dtype,
+                                       float scale, void *out, int32_t flags,
+                                       flide_stream stream) {
+  using namespace flide;
+  if (!idx || !q || !k || !v || !out) return FLIDE_ERR_SHAPE;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || past_rows < 0) return FLIDE_ERR_SHAPE;
+  if ((past_k == nullptr) != (past_v == nullptr)) return FLIDE_ERR_SHAPE;
+  if (past_k == nullptr) past_rows = 0;
+  if (idx->R < 0 || idx->R > kNoAllocMaxRequests) return FLIDE_ERR_CAPACITY;
+  if (!(flags & FLIDE_FLAG_PORTABLE) && fork_attn_tc_supported(idx, Hq, Hkv, d, dtype)) {
+    int32_t *work = noalloc_work_ptr();
+    if (!work) return FLIDE_ERR_CUDA;
+    flide_tree_index x = *idx;  // same index, work table moved to the fixed array
+    x.work = work;
+    x.work_len = kNoAllocMaxRequests + 1;
+    return fork_attn_tc(q, k, v, past_k, past_v, past_rows, &x, Hq, Hkv, scale, out,
+                        (cudaStream_t)stream);
+  }
+  // the CUDA-core kernel keeps no per-call table
+  return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,
+                            (cudaStream_t)stream);
+}

@@ -28,8 +28,8 @@ INDEX_ARRAYS = ["status", "counts", "node_start", "node_req", "depth", "anc_ptr"
 
 # every extern "C" symbol declared in include/flide.h
 SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build",
-           "flide_fork_attn", "flide_fork_gdn", "flide_state_save", "flide_state_resume",
-           "flide_strerror"]
+           "flide_fork_attn", "flide_fork_attn_noalloc", "flide_fork_gdn", "flide_state_save",
+           "flide_state_resume", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -72,6 +72,9 @@ def _lib():
         lib.flide_tree_build.restype = ctypes.c_int
         lib.flide_fork_attn.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32, F, P, I32, P]
         lib.flide_fork_attn.restype = ctypes.c_int
+        lib.flide_fork_attn_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32, F, P,
+                                                I32, P]
+        lib.flide_fork_attn_noalloc.restype = ctypes.c_int
         lib.flide_fork_gdn.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, P, P, I32, I32, P]
         lib.flide_fork_gdn.restype = ctypes.c_int
         lib.flide_state_save.argtypes = [P, P, P, P, P, I32, I32, I32, P, I32, I32, I32, P, P, P,
@@ -182,6 +185,25 @@ def fork_attn(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None,
                                   past_rows, ctypes.byref(index.c), Hq, Hkv, d, _dtype_code(q),
                                   float(scale), _ptr(out), flags, _stream(stream)),
            "flide_fork_attn")
+    return out
+
+
+def fork_attn_noalloc(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None,
+                      out=None, flags: int = 0, stream=None):
+    """flide_fork_attn_noalloc: same result as fork_attn, for callers that cannot
+    provide scratch; leaves index.c.work untouched and allocates nothing."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    past_rows = 0 if past_k is None else past_k.shape[0]
+    if past_rows == 0:
+        past_k = past_v = None
+    _check(_lib().flide_fork_attn_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(past_k), _ptr(past_v),
+                                          past_rows, ctypes.byref(index.c), Hq, Hkv, d,
+                                          _dtype_code(q), float(scale), _ptr(out), flags,
+                                          _stream(stream)),
+           "flide_fork_attn_noalloc")
     return out
 
 
