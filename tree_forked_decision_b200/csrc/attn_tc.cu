@@ -8,12 +8,13 @@
 // isolated forward pass while the shared prefix is stored and read once.
 //
 // Work decomposition.  One CTA per work item = (request, kv head, tile of
-// query tokens).  A tile packs the G = Hq/Hkv query heads of one kv head with
-// 128/G consecutive tokens into 128 MMA rows (row = token*G + head), so one
-// K/V tile in shared memory serves every query head of the group and, for a
-// branch tile, the queries of several sibling branches at once.  Tiles never
-// straddle the root/branch boundary of a request.  Key tiles come from a short
-// list of spans:
+// query tokens).  The G = Hq/Hkv query heads of one kv head are packed with
+// the tokens into MMA rows (row = token*G + head), so one K/V tile in shared
+// memory serves every query head of the group and, for a branch tile, the
+// queries of several sibling branches at once.  A tile is 256 rows, split into
+// two 128-row halves that share the K/V stream.  Tiles never straddle the
+// root/branch boundary of a request.  Key tiles come from a short list of
+// spans:
 //   past  rows of the packed checkpoint buffer      (all visible)
 //   root  the request's root segment                (branch tiles: all
 //         visible; root tiles: causal, keys up to the tile's last token)
@@ -23,17 +24,24 @@
 // Item order is (request, kv head) major with the costliest tiles first, so
 // CTAs that read the same K/V run together and share it through L2.
 //
-// CTA roles (192 threads):
-//   warps 0-3  softmax: thread = one MMA row = one TMEM lane; reads S from
-//              TMEM, masks, online softmax in the exp2 domain with lazy
-//              rescaling of O (only when the running max grows by > 2^8),
-//              writes P (bf16) to shared memory, final normalisation + store.
-//   warp 4     producer: TMA loads of Q once and of K/V tiles into a
-//              2-stage ring (128-byte swizzle).
-//   warp 5     MMA issuer: S = Q K^T into one of two TMEM buffers, then
-//              O += P V into a TMEM accumulator (tcgen05.mma kind::f16,
-//              M = N = 128, K = 16 per instruction).
-// TMEM: S0 cols [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+// CTA roles (320 threads):
+//   warps 0-3, 4-7  softmax of half 0 and half 1: thread = one MMA row = one
+//              TMEM lane; loads its S row from TMEM, masks, online softmax in
+//              the exp2 domain (O rescaled in TMEM only when the running max
+//              grows by more than 2^8), writes P as bf16 back into the S
+//              columns it has consumed, final normalisation and store.
+//   warp 8     producer: TMA loads of Q once and of K and V tiles into two
+//              2-stage rings (128-byte swizzle).
+//   warp 9     MMA issuer (one thread): per key tile j
+//                S0(j) = Q0 K^T, S1(j) = Q1 K^T      (A, B from shared memory)
+//                O0 += P0(j) V, O1 += P1(j) V        (A = P from TMEM)
+//              issued as ... PV0(j), S0(j+1), PV1(j), S1(j+1) ... so one
+//              half's softmax overlaps the other half's matrix work.  S(j+1)
+//              overwrites the columns PV(j) reads; the tensor core executes one
+//              thread's MMAs in issue order, and the commit after S(j+1)
+//              tells the softmax warps that PV(j) has finished too.
+// TMEM (512 columns): half h owns [256h, 256h+128) for S / P and
+// [256h+128, 256h+256) for O.
 // Every wait is bounded; on expiry the CTA records FLIDE_ERR_TIMEOUT, drains
 // its in-flight copies and MMAs, frees TMEM and exits.
 #include <cstddef>
@@ -49,34 +57,34 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;  // MMA rows per tile
+constexpr int BM = 128;  // MMA rows per half
 constexpr int BN = 128;  // keys per tile
-constexpr int NS = 2;    // K/V stages
 constexpr int kMaxLevels = 8;
 constexpr int kMaxSpans = 2 + kMaxLevels;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // shared-memory map, bytes from a 1024-aligned base
-constexpr int SM_Q = 0;                   // 2 slabs x [128 rows x 128 B]
-constexpr int SM_KV = 32768;              // stage s: K slab0, K slab1, V slab0, V slab1
-constexpr int SM_P = SM_KV + NS * 65536;  // 2 slabs x [128 rows x 128 B]
-constexpr int SM_BAR = SM_P + 32768;
+constexpr int SM_Q = 0;            // half h, slab s: h*32768 + s*16384  [128 rows x 128 B]
+constexpr int SM_K = 65536;        // stage st: st*32768 (+ slab*16384)
+constexpr int SM_V = 131072;       // stage st: st*32768 (+ slab*16384)
+constexpr int SM_BAR = 196608;
 constexpr int SM_MISC = SM_BAR + 256;
 constexpr int SMEM_BYTES = SM_MISC + 1024 + 1024;
 
 enum {
   B_Q = 0,
-  B_KV_FULL = 1,
-  B_KV_FREE = B_KV_FULL + NS,
-  B_S_FULL = B_KV_FREE + NS,
-  B_S_FREE = B_S_FULL + 2,
-  B_P_FULL = B_S_FREE + 2,
-  B_PV_DONE = B_P_FULL + 1,
-  B_DRAIN = B_PV_DONE + 1,
-  NUM_BARS = B_DRAIN + 1
+  B_K_FULL = 1,    // [2]
+  B_K_FREE = 3,    // [2]
+  B_V_FULL = 5,    // [2]
+  B_V_FREE = 7,    // [2]
+  B_S_FULL = 9,    // [2 halves]
+  B_P_FULL = 11,   // [2 halves], 4 warp arrivals
+  B_O_FULL = 13,
+  B_DRAIN = 14,
+  NUM_BARS = 15
 };
 
 enum { SRC_STREAM = 0, SRC_PAST = 1 };
@@ -98,8 +106,8 @@ struct Misc {
 struct TcParams {
   flide_tree_index x;
   __nv_bfloat16 *out;
-  int Hq, Hkv, G, mtok, has_past;
-  float qk_log2;  // scale * log2(e)
+  int Hq, Hkv, G, mtok, has_past;  // mtok = tokens per 128-row half
+  float qk_log2;                   // scale * log2(e)
 };
 
 __device__ __forceinline__ int upper_bound_dev(const int32_t *a, int n, int key) {
@@ -111,9 +119,9 @@ __device__ __forceinline__ int upper_bound_dev(const int32_t *a, int n, int key)
   return lo;
 }
 
-// Item counts per request: Hkv * (branch tiles + root tiles), prefix-summed
-// into work[0..R].
-__global__ void attn_items_kernel(flide_tree_index x, int Hkv, int mtok) {
+// Item counts per request: Hkv * (branch tiles + root tiles) of `ttok`
+// tokens each, prefix-summed into work[0..R].
+__global__ void attn_items_kernel(flide_tree_index x, int Hkv, int ttok) {
   __shared__ int scratch[40];
   if (failed(x.status)) return;
   const int R = x.R;
@@ -125,7 +133,7 @@ __global__ void attn_items_kernel(flide_tree_index x, int Hkv, int mtok) {
       const int n0 = x.req_node[r], n1 = x.req_node[r + 1];
       if (n1 > n0) {
         const int rs = x.node_start[n0], re = x.node_start[n0 + 1], end = x.node_start[n1];
-        cnt = Hkv * ((re - rs + mtok - 1) / mtok + (end - re + mtok - 1) / mtok);
+        cnt = Hkv * ((re - rs + ttok - 1) / ttok + (end - re + ttok - 1) / ttok);
       }
     }
     int tot;
@@ -141,7 +149,7 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
   const flide_tree_index &x = p.x;
   const int R = x.R;
   const int item = blockIdx.x;
-  int valid = !failed(x.status) && item < x.work[R];
+  const int valid = !failed(x.status) && item < x.work[R];
   if (!valid) {
     if (lane == 0) ms.valid = 0;
     return;
@@ -152,20 +160,20 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
   const int root_start = x.node_start[root];
   const int br_start = x.node_start[root + 1];
   const int req_end = x.node_start[x.req_node[r + 1]];
-  const int mtok = p.mtok;
-  const int nrt = (br_start - root_start + mtok - 1) / mtok;
-  const int nbt = (req_end - br_start + mtok - 1) / mtok;
+  const int ttok = 2 * p.mtok;
+  const int nrt = (br_start - root_start + ttok - 1) / ttok;
+  const int nbt = (req_end - br_start + ttok - 1) / ttok;
   const int per = nrt + nbt;
   const int hk = local / per, w = local % per;
   const bool branch = w < nbt;
   int t0, ntok;
   if (branch) {
-    t0 = br_start + w * mtok;
-    ntok = min(mtok, req_end - t0);
+    t0 = br_start + w * ttok;
+    ntok = min(ttok, req_end - t0);
   } else {
     const int i = nrt - 1 - (w - nbt);
-    t0 = root_start + i * mtok;
-    ntok = min(mtok, br_start - t0);
+    t0 = root_start + i * ttok;
+    ntok = min(ttok, br_start - t0);
   }
   Span sp[kMaxSpans];
   int ns = 0;
@@ -218,6 +226,14 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
   }
 }
 
+// (span, offset) of key tile j; spans are few, a linear walk is cheap
+__device__ __forceinline__ void tile_at(const Misc &ms, int j, Span &sp, int &off) {
+  int s = 0;
+  while (s + 1 < ms.n_spans && ms.spans[s + 1].tile0 <= j) ++s;
+  sp = ms.spans[s];
+  off = (j - sp.tile0) * BN;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_pk,
@@ -231,18 +247,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const flide_tree_index &x = p.x;
   auto bar = [&](int i) -> uint32_t { return sb + SM_BAR + 8 * i; };
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
-      for (int i = 0; i < NUM_BARS; ++i) {
-        uint32_t cnt = 1;
-        if (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) cnt = 4;
-        mbar_init(bar(i), cnt);
-      }
+      for (int i = 0; i < NUM_BARS; ++i)
+        mbar_init(bar(i), (i == B_P_FULL || i == B_P_FULL + 1) ? 4u : 1u);
       ms.abort = 0;
       fence_mbar_init();
     }
     decode_item(p, ms, lane);
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     tmem_alloc(sb + SM_MISC + (uint32_t)offsetof(Misc, tmem_base), 512);
     tmem_relinquish();
   }
@@ -252,223 +265,221 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const uint32_t tmem = ms.tmem_base;
 
   if (ms.valid) {
-    const int n_spans = ms.n_spans, n_tiles = ms.n_tiles;
+    const int n_tiles = ms.n_tiles;
     const int hk = ms.hk, t0 = ms.t0, ntok = ms.ntok;
-    if (warp == 4) {
+    if (warp == 8) {
       // ------------------------------------------------------------ producer
       if (lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(bar(B_Q), BM * 128 * 2);
-        tma_load_3d(sb + SM_Q, &tm_q, bar(B_Q), 0, hk * p.G, t0);
-        tma_load_3d(sb + SM_Q + 16384, &tm_q, bar(B_Q), 64, hk * p.G, t0);
-        int j = 0;
+        mbar_arrive_expect_tx(bar(B_Q), 2 * BM * 128 * 2);
+        for (int h = 0; h < 2; ++h)
+          for (int s = 0; s < 2; ++s)
+            tma_load_3d(sb + SM_Q + h * 32768 + s * 16384, &tm_q, bar(B_Q), 64 * s, hk * p.G,
+                        t0 + h * p.mtok);
+        int jk = 0, jv = 0;  // tiles issued
         bool ok = true;
-        for (int s = 0; s < n_spans && ok; ++s) {
-          const Span sp = ms.spans[s];
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          Span sp;
+          int off;
+          tile_at(ms, j, sp, off);
           const CUtensorMap *mk = sp.src == SRC_PAST ? &tm_pk : &tm_k;
           const CUtensorMap *mv = sp.src == SRC_PAST ? &tm_pv : &tm_v;
-          for (int off = 0; off < sp.len; off += BN, ++j) {
-            const int st = j % NS;
-            if (j >= NS && !mbar_wait(bar(B_KV_FREE + st), ((j / NS) - 1) & 1, abort_flag, kTimeoutNs)) {
-              ok = false;
-              break;
-            }
-            const uint32_t dst = sb + SM_KV + st * 65536;
-            const int row = sp.start + off;
-            mbar_arrive_expect_tx(bar(B_KV_FULL + st), 65536);
-            tma_load_3d(dst, mk, bar(B_KV_FULL + st), 0, hk, row);
-            tma_load_3d(dst + 16384, mk, bar(B_KV_FULL + st), 64, hk, row);
-            tma_load_3d(dst + 32768, mv, bar(B_KV_FULL + st), 0, hk, row);
-            tma_load_3d(dst + 49152, mv, bar(B_KV_FULL + st), 64, hk, row);
+          const int row = sp.start + off;
+          const int st = j & 1;
+          if (j >= 2 && !mbar_wait(bar(B_K_FREE + st), ((j >> 1) - 1) & 1, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
           }
+          mbar_arrive_expect_tx(bar(B_K_FULL + st), BN * 128 * 2);
+          tma_load_3d(sb + SM_K + st * 32768, mk, bar(B_K_FULL + st), 0, hk, row);
+          tma_load_3d(sb + SM_K + st * 32768 + 16384, mk, bar(B_K_FULL + st), 64, hk, row);
+          ++jk;
+          if (j >= 2 && !mbar_wait(bar(B_V_FREE + st), ((j >> 1) - 1) & 1, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(B_V_FULL + st), BN * 128 * 2);
+          tma_load_3d(sb + SM_V + st * 32768, mv, bar(B_V_FULL + st), 0, hk, row);
+          tma_load_3d(sb + SM_V + st * 32768 + 16384, mv, bar(B_V_FULL + st), 64, hk, row);
+          ++jv;
         }
         if (!ok) {
           // drain the copies still in flight into this CTA's shared memory
           mbar_wait(bar(B_Q), 0, abort_flag, kTimeoutNs, false);
-          for (int jj = max(0, j - NS); jj < j; ++jj)
-            mbar_wait(bar(B_KV_FULL + jj % NS), (jj / NS) & 1, abort_flag, kTimeoutNs, false);
+          for (int jj = max(0, jk - 2); jj < jk; ++jj)
+            mbar_wait(bar(B_K_FULL + (jj & 1)), (jj >> 1) & 1, abort_flag, kTimeoutNs, false);
+          for (int jj = max(0, jv - 2); jj < jv; ++jj)
+            mbar_wait(bar(B_V_FULL + (jj & 1)), (jj >> 1) & 1, abort_flag, kTimeoutNs, false);
         }
       }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
       // ------------------------------------------------------------ MMA
       if (lane == 0) {
         constexpr uint32_t id_s = idesc_bf16(BM, BN, false);
         constexpr uint32_t id_pv = idesc_bf16(BM, 128, true);
-        bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kTimeoutNs);
-        auto do_pv = [&](int i) -> bool {
-          if (!mbar_wait(bar(B_P_FULL), i & 1, abort_flag, kTimeoutNs)) return false;
-          tc_fence_after();
-          const int st = i % NS;
-          const uint32_t vb = sb + SM_KV + st * 65536 + 32768;
+        auto qk = [&](int h, int st) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sdesc_sw128(sb + SM_P + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(vb + kk * 2048, 16384, 1024);
-            mma_bf16(tmem + 256, a, b, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t a = sdesc_sw128(sb + SM_Q + h * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sb + SM_K + st * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            mma_bf16(tmem + h * 256, a, b, id_s, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(B_KV_FREE + st));
-          mma_commit(bar(B_PV_DONE));
-          return true;
         };
-        int j = 0;
-        for (; ok && j < n_tiles; ++j) {
-          const int st = j % NS;
-          if (!mbar_wait(bar(B_KV_FULL + st), (j / NS) & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
-          if (j >= 2 && !mbar_wait(bar(B_S_FREE + (j & 1)), ((j >> 1) - 1) & 1, abort_flag, kTimeoutNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t kb = sb + SM_KV + st * 65536;
+        auto pv = [&](int h, int st, bool acc) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sdesc_sw128(sb + SM_Q + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(kb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            mma_bf16(tmem + (j & 1) * 128, a, b, id_s, kk > 0 ? 1u : 0u);
+            const uint64_t b = sdesc_sw128(sb + SM_V + st * 32768 + kk * 2048, 16384, 1024);
+            mma_bf16_ts(tmem + h * 256 + 128, tmem + h * 256 + kk * 8, b, id_pv,
+                        (acc || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar(B_S_FULL + (j & 1)));
-          if (j >= 1 && !do_pv(j - 1)) { ok = false; break; }
+        };
+        bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kTimeoutNs) &&
+                  mbar_wait(bar(B_K_FULL), 0, abort_flag, kTimeoutNs);
+        if (ok) {
+          tc_fence_after();
+          qk(0, 0);
+          mma_commit(bar(B_S_FULL + 0));
+          qk(1, 0);
+          mma_commit(bar(B_S_FULL + 1));
+          mma_commit(bar(B_K_FREE + 0));
         }
-        if (ok) do_pv(n_tiles - 1);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int sv = j & 1, sk = (j + 1) & 1;
+          const bool more = j + 1 < n_tiles;
+          if (!mbar_wait(bar(B_V_FULL + sv), (j >> 1) & 1, abort_flag, kTimeoutNs) ||
+              !mbar_wait(bar(B_P_FULL + 0), j & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
+          tc_fence_after();
+          pv(0, sv, j > 0);
+          if (more) {
+            if (!mbar_wait(bar(B_K_FULL + sk), ((j + 1) >> 1) & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
+            tc_fence_after();
+            qk(0, sk);
+            mma_commit(bar(B_S_FULL + 0));
+          }
+          if (!mbar_wait(bar(B_P_FULL + 1), j & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
+          tc_fence_after();
+          pv(1, sv, j > 0);
+          mma_commit(bar(B_V_FREE + sv));
+          if (more) {
+            qk(1, sk);
+            mma_commit(bar(B_S_FULL + 1));
+            mma_commit(bar(B_K_FREE + sk));
+          }
+        }
+        if (ok) mma_commit(bar(B_O_FULL));
         // all MMAs issued by this thread complete before TMEM is released
         mma_commit(bar(B_DRAIN));
         mbar_wait(bar(B_DRAIN), 0, abort_flag, kTimeoutNs, false);
       }
     } else {
       // ------------------------------------------------------------ softmax
-      const int row = warp * 32 + lane;
-      const int tokr = row / p.G, g = row % p.G;
+      const int h = warp >> 2;                      // half
+      const int row = (warp & 3) * 32 + lane;       // TMEM lane = MMA row in the half
+      const int tokr = h * p.mtok + row / p.G, g = row % p.G;
       const bool valid_row = tokr < ntok;
       const int t = t0 + tokr;
       const int row_node = valid_row ? x.token_node[t] : -1;
       const int row_depth = valid_row ? x.depth[row_node] : -1;
       const int row_anc = valid_row ? x.anc_ptr[row_node] : 0;
-      const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+      const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lanes
+      const uint32_t t_s = tl + h * 256, t_o = tl + h * 256 + 128;
+      const float c = p.qk_log2;
       float m_used = -INFINITY, l = 0.f;
-      uint8_t *P = smem + SM_P;
       bool ok = true;
-      int j = 0;
-      for (int s = 0; s < n_spans && ok; ++s) {
-        const Span sp = ms.spans[s];
-        const int a_row = (sp.kind == KIND_TREE && valid_row && row_depth >= sp.level)
-                              ? x.anc_node[row_anc + sp.level]
-                              : -2;
-        for (int off = 0; off < sp.len; off += BN, ++j) {
-          const int buf = j & 1;
-          // every lane waits; the warp proceeds only if all lanes saw the phase
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + buf), (j >> 1) & 1, abort_flag, kTimeoutNs))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          float sv[BN];
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            uint32_t rr[32];
-            tmem_ld32(lane_base + buf * 128 + c4 * 32, rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[c4 * 32 + i] = __uint_as_float(rr[i]);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_S_FREE + buf));
-          const int rem = sp.len - off;
-          if (sp.kind != KIND_FULL || rem < BN) {
-            const int key0 = sp.start + off;
-#pragma unroll
-            for (int c = 0; c < BN; ++c) {
-              bool vis = c < rem;
-              const int key = key0 + c;
-              if (sp.kind == KIND_CAUSAL) vis = vis && key <= t;
-              if (sp.kind == KIND_TREE) {
-                const int kn = vis ? x.token_node[key] : -1;
-                vis = vis && kn == a_row && (kn != row_node || key <= t);
-              }
-              if (!vis) sv[c] = -INFINITY;
-            }
-          }
-          float smax = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < BN; ++c) smax = fmaxf(smax, sv[c]);
-          const float mt = smax * p.qk_log2;
-          if (j == 0) {
-            m_used = mt;
-          } else {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(B_PV_DONE), (j - 1) & 1, abort_flag, kTimeoutNs))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const bool need = mt > m_used + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, need)) {
-              const float f = need ? exp2f(m_used - mt) : 1.f;
-#pragma unroll
-              for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t rr[32];
-                tmem_ld32(lane_base + 256 + c4 * 32, rr);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
-                tmem_st32(lane_base + 256 + c4 * 32, rr);
-              }
-              l *= f;
-              if (need) m_used = mt;
-            }
-          }
-          const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-          float rs = 0.f;
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            sv[c] = exp2f(fmaf(sv[c], p.qk_log2, -m_sub));
-            rs += sv[c];
-          }
-          l += rs;
-#pragma unroll
-          for (int sl = 0; sl < 2; ++sl) {
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const int c0 = sl * 64 + ch * 8;
-              uint4 pk;
-              __nv_bfloat162 b0 = __floats2bfloat162_rn(sv[c0 + 0], sv[c0 + 1]);
-              __nv_bfloat162 b1 = __floats2bfloat162_rn(sv[c0 + 2], sv[c0 + 3]);
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[c0 + 4], sv[c0 + 5]);
-              __nv_bfloat162 b3 = __floats2bfloat162_rn(sv[c0 + 6], sv[c0 + 7]);
-              pk.x = *reinterpret_cast<uint32_t *>(&b0);
-              pk.y = *reinterpret_cast<uint32_t *>(&b1);
-              pk.z = *reinterpret_cast<uint32_t *>(&b2);
-              pk.w = *reinterpret_cast<uint32_t *>(&b3);
-              *reinterpret_cast<uint4 *>(P + sl * 16384 + row * 128 + ((ch ^ (row & 7)) << 4)) = pk;
-            }
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_P_FULL));
+      for (int j = 0; j < n_tiles; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + h), j & 1, abort_flag, kTimeoutNs))) {
+          ok = false;
+          break;
         }
-      }
-      if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV_DONE), (n_tiles - 1) & 1, abort_flag, kTimeoutNs))) {
         tc_fence_after();
-        const float inv = 1.f / l;
-        __nv_bfloat16 *o = p.out + ((size_t)t * p.Hq + hk * p.G + g) * 128;
+        Span sp;
+        int off;
+        tile_at(ms, j, sp, off);
+        uint32_t sr[128];
+        tmem_ld128(t_s, sr);
+        float sv[128];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t rr[32];
-          tmem_ld32(lane_base + 256 + c4 * 32, rr);
-          if (valid_row) {
+        for (int i = 0; i < 128; ++i) sv[i] = __uint_as_float(sr[i]);
+        const int rem = sp.len - off;
+        if (sp.kind != KIND_FULL || rem < BN) {
+          const int key0 = sp.start + off;
+          const int a_row = (sp.kind == KIND_TREE && valid_row && row_depth >= sp.level)
+                                ? x.anc_node[row_anc + sp.level]
+                                : -2;
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-              uint4 pk;
-              __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(rr[q8 * 8 + 0]) * inv, __uint_as_float(rr[q8 * 8 + 1]) * inv);
-              __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(rr[q8 * 8 + 2]) * inv, __uint_as_float(rr[q8 * 8 + 3]) * inv);
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(rr[q8 * 8 + 4]) * inv, __uint_as_float(rr[q8 * 8 + 5]) * inv);
-              __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(rr[q8 * 8 + 6]) * inv, __uint_as_float(rr[q8 * 8 + 7]) * inv);
-              pk.x = *reinterpret_cast<uint32_t *>(&b0);
-              pk.y = *reinterpret_cast<uint32_t *>(&b1);
-              pk.z = *reinterpret_cast<uint32_t *>(&b2);
-              pk.w = *reinterpret_cast<uint32_t *>(&b3);
-              *reinterpret_cast<uint4 *>(o + c4 * 32 + q8 * 8) = pk;
+          for (int i = 0; i < BN; ++i) {
+            bool vis = i < rem;
+            const int key = key0 + i;
+            if (sp.kind == KIND_CAUSAL) vis = vis && key <= t;
+            if (sp.kind == KIND_TREE) {
+              const int kn = vis ? x.token_node[key] : -1;
+              vis = vis && kn == a_row && (kn != row_node || key <= t);
             }
+            if (!vis) sv[i] = -INFINITY;
+          }
+        }
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+        for (int i = 8; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+        const float smax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mt = smax * c;
+        if (j == 0) {
+          m_used = mt;
+        } else {
+          // PV(j-1) of this half is complete (it precedes S(j) in issue order)
+          const bool need = mt > m_used + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float f = need ? exp2f(m_used - mt) : 1.f;
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+              uint32_t r32[32];
+              tmem_ld32(t_o + 32 * c4, r32);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * f);
+              tmem_st32(t_o + 32 * c4, r32);
+            }
+            l *= f;
+            if (need) m_used = mt;
+          }
+        }
+        const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+        float ps[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ps[i] = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < BN; i += 2) {
+          const float e0 = ex2_approx(fmaf(sv[i], c, -m_sub));
+          const float e1 = ex2_approx(fmaf(sv[i + 1], c, -m_sub));
+          ps[(i >> 1) & 7] += e0 + e1;
+          pk[i >> 1] = pack_bf16x2(e0, e1);
+        }
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        tmem_st64(t_s, pk);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_P_FULL + h));
+      }
+      if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL), 0, abort_flag, kTimeoutNs))) {
+        tc_fence_after();
+        uint32_t orr[128];
+        tmem_ld128(t_o, orr);
+        if (valid_row) {
+          const float inv = 1.f / l;
+          __nv_bfloat16 *o = p.out + ((size_t)t * p.Hq + hk * p.G + g) * 128;
+#pragma unroll
+          for (int q8 = 0; q8 < 16; ++q8) {
+            uint4 v4;
+            v4.x = pack_bf16x2(__uint_as_float(orr[q8 * 8 + 0]) * inv, __uint_as_float(orr[q8 * 8 + 1]) * inv);
+            v4.y = pack_bf16x2(__uint_as_float(orr[q8 * 8 + 2]) * inv, __uint_as_float(orr[q8 * 8 + 3]) * inv);
+            v4.z = pack_bf16x2(__uint_as_float(orr[q8 * 8 + 4]) * inv, __uint_as_float(orr[q8 * 8 + 5]) * inv);
+            v4.w = pack_bf16x2(__uint_as_float(orr[q8 * 8 + 6]) * inv, __uint_as_float(orr[q8 * 8 + 7]) * inv);
+            *reinterpret_cast<uint4 *>(o + q8 * 8) = v4;
           }
         }
       }
@@ -477,7 +488,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   if (ms.valid && ms.abort && threadIdx.x == 0) set_status(x.status, FLIDE_ERR_TIMEOUT);
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -532,7 +543,7 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
                  int past_rows, const flide_tree_index *x, int Hq, int Hkv, float scale,
                  void *out, cudaStream_t s) {
   const int G = Hq / Hkv;
-  const int mtok = BM / G;
+  const int mtok = BM / G;  // tokens per 128-row half; a tile is 2*mtok tokens
   CUtensorMap mq, mk, mv, mpk, mpv;
   const long T = x->T > 0 ? x->T : 1;
   if (!make_map(&mq, q, Hq, T, G, mtok)) return FLIDE_ERR_CUDA;
@@ -552,7 +563,7 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
       return FLIDE_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  attn_items_kernel<<<1, 1024, 0, s>>>(*x, Hkv, mtok);
+  attn_items_kernel<<<1, 1024, 0, s>>>(*x, Hkv, 2 * mtok);
   FLIDE_LAUNCH_CHECK();
   TcParams prm;
   prm.x = *x;
@@ -563,7 +574,7 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
   prm.mtok = mtok;
   prm.has_past = has_past ? 1 : 0;
   prm.qk_log2 = scale * kLog2e;
-  const long grid = (long)Hkv * ((x->T + mtok - 1) / mtok + 2L * x->R);
+  const long grid = (long)Hkv * ((x->T + 2 * mtok - 1) / (2 * mtok) + 2L * x->R);
   if (grid <= 0) return FLIDE_OK;
   if (grid > 0x7fffffffL) return FLIDE_ERR_CAPACITY;
   attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mpk, mpv, prm);
