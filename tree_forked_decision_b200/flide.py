@@ -161,6 +161,16 @@ class DeviceTree:
             self.parent = torch.full((1,), -1, dtype=torch.int32, device=device)
             self.seg_len = torch.zeros(1, dtype=torch.int32, device=device)
 
+    @classmethod
+    def from_buffers(cls, req_node_ptr, parent, seg_len, past_len, N: int, T: int,
+                     max_depth: int) -> "DeviceTree":
+        """Wraps preallocated int32 device buffers (capacities N, T) without copying."""
+        t = cls.__new__(cls)
+        t.req_node_ptr, t.parent, t.seg_len, t.past_len = req_node_ptr, parent, seg_len, past_len
+        t.R = req_node_ptr.shape[0] - 1
+        t.N, t.T, t.max_depth = int(N), int(T), int(max_depth)
+        return t
+
     def desc(self) -> TreeDesc:
         return TreeDesc(self.R, self.N, self.T, self.max_depth, self.req_node_ptr.data_ptr(),
                         self.parent.data_ptr(), self.seg_len.data_ptr(), self.past_len.data_ptr())
