@@ -23,14 +23,23 @@ EDGE_TREES = {
 }
 
 
+@pytest.mark.parametrize("flags", [0, flide.FLAG_PORTABLE], ids=["tc", "portable"])
 @pytest.mark.parametrize("case", sorted(EDGE_TREES))
-def test_edge_attention_and_gdn(case):
+def test_edge_attention_and_gdn(case, flags):
     tree = EDGE_TREES[case]()
     rng = np.random.default_rng(3)
     a = inputs.attn_inputs(tree, 8, 2, 128, torch.bfloat16, rng)
-    got, scale = run_attn(tree, a)
+    got, scale = run_attn(tree, a, flags=flags)
     assert np.all(np.isfinite(got))
     assert_close(got, oracle_attn(tree, a, scale), torch.bfloat16)
+    g = inputs.gdn_inputs(tree, 2, 128, 128, torch.bfloat16, rng, gate_scale=0.1)
+    gg, _, _ = run_gdn(tree, g, flags=flags)
+    assert_close(gg, oracle_gdn(tree, g), torch.bfloat16)
+
+
+def test_edge_gdn_small_head_dims():
+    tree = EDGE_TREES["zero_token_root_with_past"]()
+    rng = np.random.default_rng(4)
     g = inputs.gdn_inputs(tree, 2, 64, 64, torch.bfloat16, rng, gate_scale=0.1)
     gg, _, _ = run_gdn(tree, g)
     assert_close(gg, oracle_gdn(tree, g), torch.bfloat16)

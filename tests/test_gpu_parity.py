@@ -193,13 +193,31 @@ def test_gdn_fp32_random_trees(seed):
     assert_close(got, oracle_gdn(tree, g), torch.float32)
 
 
-@pytest.mark.parametrize("seed", range(2))
-def test_gdn_bf16_leveled(seed):
+@pytest.mark.parametrize("flags", [0, flide.FLAG_PORTABLE], ids=["tc", "portable"])
+@pytest.mark.parametrize("seed", range(3))
+def test_gdn_bf16_leveled(seed, flags):
     rng = np.random.default_rng(800 + seed)
     tree = inputs.leveled_tree(rng, 3, depth_range=(1, 3), options_range=(3, 30),
                                prefix_range=(60, 300), n_resume=1)
     g = inputs.gdn_inputs(tree, 4, 128, 128, torch.bfloat16, rng, gate_scale=0.1)
-    got, _, _ = run_gdn(tree, g)
+    got, node_state, idx = run_gdn(tree, g, flags=flags)
+    want, states = oracle_gdn(tree, g, want_states=True)
+    assert_close(got, want, torch.bfloat16)
+    # saved end states of roots and inner nodes
+    slot = idx.array("state_slot", tree.N).cpu().numpy()
+    ns = node_state.cpu().numpy()
+    for n in range(tree.N):
+        if slot[n] >= 0:
+            err = np.abs(ns[slot[n]] - states[n]).max()
+            assert err <= 2e-2, (n, err)
+
+
+@pytest.mark.parametrize("flags", [0, flide.FLAG_PORTABLE], ids=["tc", "portable"])
+def test_gdn_bf16_strong_gates_long_prefix(flags):
+    # gate scale 1 (alpha ~ 0.45 per token) over a prefix of many chunks
+    tree = inputs.fanout_tree(2, 700, 9, 13, past=5)
+    g = inputs.gdn_inputs(tree, 2, 128, 128, torch.bfloat16, np.random.default_rng(9), gate_scale=1.0)
+    got, _, _ = run_gdn(tree, g, flags=flags)
     assert_close(got, oracle_gdn(tree, g), torch.bfloat16)
 
 

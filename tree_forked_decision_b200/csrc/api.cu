@@ -16,6 +16,10 @@ bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, i
 int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, const void *pv,
                  int past_rows, const flide_tree_index *x, int Hq, int Hkv, float scale,
                  void *out, cudaStream_t s);
+bool fork_gdn_tc_supported(int dk, int dv, int dtype);
+int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                const float *state_in, const flide_tree_index *x, int H, void *out,
+                float *node_state, int n_slots, cudaStream_t s);
 int fork_gdn_portable(const void *q, const void *k, const void *v, const float *g,
                       const float *beta, const float *state_in, const flide_tree_index *x,
                       int H, int dk, int dv, int dtype, void *out, float *node_state,
@@ -34,8 +38,11 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
-// int32 entries of the per-call scratch `work`
-int64_t work_entries(int32_t R) { return 4 * (int64_t)(R + 1) + 1024; }
+// int32 entries of the per-call scratch `work`: the attention's per-request
+// item table and the GDN's per-level node groups (see their kernels)
+int64_t work_entries(int32_t R, int32_t N) {
+  return 4 * (int64_t)(R + 1) + 3 * (int64_t)(N + 1) + 1024;
+}
 
 struct Layout {
   size_t off[18];
@@ -61,7 +68,7 @@ bool layout(int32_t R, int32_t N, int32_t T, int32_t D, Layout *L) {
                          N,
                          N,
                          (int64_t)R + 1,
-                         work_entries(R)};
+                         work_entries(R, N)};
   size_t o = 0;
   for (int i = 0; i < 17; ++i) {
     L->off[i] = o;
@@ -102,7 +109,7 @@ int flide_tree_index_init(flide_tree_index *idx, void *dev_buf, size_t bytes, in
   idx->N = N;
   idx->T = T;
   idx->max_depth = max_depth;
-  idx->work_len = work_entries(R);
+  idx->work_len = work_entries(R, N);
   return FLIDE_OK;
 }
 
@@ -129,9 +136,11 @@ int flide_fork_gdn(const void *q, const void *k, const void *v, const float *g,
                    const float *beta, const float *state_in, flide_tree_index *idx, int32_t H,
                    int32_t dk, int32_t dv, int32_t dtype, void *out, float *node_state,
                    int32_t n_state_slots, int32_t flags, flide_stream stream) {
-  (void)flags;
   if (!idx || !q || !k || !v || !g || !beta || !out || !node_state) return FLIDE_ERR_SHAPE;
   if (H <= 0 || n_state_slots <= 0) return FLIDE_ERR_SHAPE;
+  if (!(flags & FLIDE_FLAG_PORTABLE) && fork_gdn_tc_supported(dk, dv, dtype))
+    return fork_gdn_tc(q, k, v, g, beta, state_in, idx, H, out, node_state, n_state_slots,
+                       (cudaStream_t)stream);
   return fork_gdn_portable(q, k, v, g, beta, state_in, idx, H, dk, dv, dtype, out, node_state,
                            n_state_slots, (cudaStream_t)stream);
 }

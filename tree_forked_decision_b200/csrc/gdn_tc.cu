@@ -1,0 +1,684 @@
+// gdn_tc.cu -- Gated DeltaNet fork scan on the 5th-generation tensor cores
+// (sm_100a): bf16 q/k/v, dk = dv = 128, fp32 state and accumulation.
+//
+// Per head the state S (dv x dk) follows the gated delta rule
+//   S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t.
+// Forking (kongchang.com article on Flide, Gated DeltaNet box; techfi24.com,
+// "Exact State Forking"): every root scans from its request's state_in (the
+// prefix, once) and saves its end state; every other node starts from its
+// parent's saved end state; nodes with children save their end state too.
+// One launch per tree level, ordered by the stream.
+//
+// Chunked form used here (C = 64 tokens; the same sums grouped differently,
+// equal in exact arithmetic).  With G_i the running sum of g inside the chunk,
+// gamma_i = exp(G_i) and S0 the state before the chunk,
+//   A_ij = b_i (gamma_i/gamma_j) k_i.k_j  (j < i),   T = (I + A)^-1,
+//   W = T diag(b gamma) K,   U = T diag(b) V,   Delta = U - W S0^T,
+//   O = diag(gamma) Q S0^T + (M o QK^T) Delta,  M_ij = gamma_i/gamma_j (j <= i),
+//   S_end = gamma_last S0 + Delta^T diag(gamma_last/gamma) K.
+// Tensor-core products, all M = 128 x N = 128 with a K-major shared-memory A
+// operand (rows = tokens padded to 128, or state rows):
+//   R1 = [K;Q] [K;Q]^T     -> KK^T (rows 0-63) and QK^T (rows 64-127)
+//   R2 = T' K,  R3 = T'' V -> W and U (T' = T diag(b gamma), T'' = T diag(b))
+//   R3 += (-W) S0^T        -> Delta         R1 = [K;Q] S0^T -> Q S0^T (rows 64-127)
+//   R2 = (M o QK^T) Delta  -> rows 64-127   S += Delta'^T K  (Delta' = Delta gamma_last/gamma)
+// T is solved in fp32 on CUDA cores (one column per thread).  The fp32 state
+// lives in TMEM for the whole scan; a bf16 copy is the operand for a chunk.
+//
+// Work items (built per level by gdn_groups_kernel): a root, an inner node or
+// a node longer than one chunk is a "scan" item (its chunks in order, state
+// carried in TMEM, end state saved when the node has a slot); runs of
+// consecutive sibling leaves that fit one chunk are packed into one item with
+// a block-diagonal mask, so no leaf sees another.  Items x heads are spread
+// over a persistent grid of one CTA per SM.  Every wait is bounded (2 s).
+#include <cstddef>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace flide {
+namespace {
+
+using namespace sm100;
+
+constexpr int C = 64;    // tokens per chunk
+constexpr int D = 128;   // dk = dv
+constexpr int kThreads = 128;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+// shared-memory map, bytes from a 1024-aligned base
+constexpr int SM_KQ = 0;        // stage s: s*32768; slab b (64 dims): +b*16384; K rows 0-63, Q rows 64-127
+constexpr int SM_V = 65536;     // stage s: s*16384; slab b: +b*8192; rows 0-63
+constexpr int SM_S0 = 98304;    // bf16 S0 [128 dv rows][dk], K-major, 2 slabs x 16 KB; then
+                                //   Delta [64 token rows][dv] MN-major (2 slabs x 8 KB) at +0 and
+                                //   Delta'^T [128 dv rows][64 tokens] K-major at +16384
+constexpr int SM_TA = 131072;   // T' and T'' [128 rows][64] K-major (16 KB each); then
+                                //   -W [128 rows][dk] K-major (2 slabs x 16 KB)
+constexpr int SM_PM = 163840;   // (M o QK^T) [128 rows][64] K-major, token rows at 64-127
+constexpr int SM_A = 180224;    // fp32 A [64][65]
+constexpr int A_LD = 65;
+constexpr int SM_SCAL = SM_A + C * A_LD * 4;  // beta, G, gamma, seg: 4 x 64 words
+constexpr int SM_BAR = SM_SCAL + 4 * C * 4;
+constexpr int SM_MISC = SM_BAR + 64;
+constexpr int SMEM_BYTES = SM_MISC + 64 + 1024;
+
+// TMEM column regions (128 each)
+constexpr uint32_t R_S = 0, R1 = 128, R2 = 256, R3 = 384;
+
+enum { B_FULL = 0, B_MMA = 2, NUM_BARS = 3 };
+
+struct GdnTcParams {
+  flide_tree_index x;
+  const float *g, *beta, *state_in;
+  __nv_bfloat16 *out;
+  float *node_state;
+  int H, n_slots, level, goff;
+};
+
+// work[goff] = number of groups; work[goff+1+g] = first level position of
+// group g; work[goff+2+N+g] = its node count.
+__device__ __forceinline__ int *groups_n(const flide_tree_index &x, int goff) { return x.work + goff; }
+__device__ __forceinline__ int *groups_start(const flide_tree_index &x, int goff) {
+  return x.work + goff + 1;
+}
+__device__ __forceinline__ int *groups_count(const flide_tree_index &x, int goff) {
+  return x.work + goff + 2 + x.N;
+}
+
+// Groups the nodes of one level: a root, a node with a state slot or a node
+// longer than a chunk is alone; consecutive leaves (consecutive ids) with the
+// same parent are packed greedily while they fit one chunk.
+__global__ void gdn_groups_kernel(flide_tree_index x, int level, int goff) {
+  __shared__ int scratch[40];
+  int *flag = groups_count(x, goff);  // temporary flags, then counts
+  int *gstart = groups_start(x, goff);
+  if (failed(x.status)) {
+    if (threadIdx.x == 0) *groups_n(x, goff) = 0;
+    return;
+  }
+  const int L0 = x.level_ptr[level], n = x.level_ptr[level + 1] - L0;
+  auto seg = [&](int node) { return x.node_start[node + 1] - x.node_start[node]; };
+  auto alone = [&](int node) { return level == 0 || x.state_slot[node] >= 0 || seg(node) > C; };
+  auto parent_of = [&](int node) { return x.anc_node[x.anc_ptr[node + 1] - 2]; };
+  // 1: run starts
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const int node = x.level_node[L0 + k];
+    int f = 1;
+    if (k > 0) {
+      const int prev = x.level_node[L0 + k - 1];
+      f = alone(node) || alone(prev) || prev + 1 != node || parent_of(prev) != parent_of(node);
+    }
+    flag[k] = f;
+  }
+  __syncthreads();
+  // 2: one thread per run packs it greedily by tokens
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    if (!flag[k]) continue;
+    int tok = 0;
+    for (int e = k; e < n && (e == k || !flag[e]); ++e) {
+      const int sl = seg(x.level_node[L0 + e]);
+      if (e > k && tok + sl > C) {
+        flag[e] = 2;  // starts a new group inside the run
+        tok = 0;
+      }
+      tok += sl;
+    }
+  }
+  __syncthreads();
+  // 3: compact the group starts
+  int carry = 0;
+  for (int b = 0; b < n; b += blockDim.x) {
+    const int k = b + threadIdx.x;
+    const int f = (k < n && flag[k] != 0) ? 1 : 0;
+    int tot;
+    const int ex = block_excl_scan(f, scratch, &tot);
+    if (f) gstart[carry + ex] = k;
+    carry += tot;
+  }
+  __syncthreads();
+  // 4: counts
+  for (int g = threadIdx.x; g < carry; g += blockDim.x)
+    flag[g] = (g + 1 < carry ? gstart[g + 1] : n) - gstart[g];
+  if (threadIdx.x == 0) *groups_n(x, goff) = carry;
+}
+
+// Self-check: records the first failed bounds check (site, value) in the
+// index's spare count slots 12-13 and the status word; the caller skips the
+// access.
+__device__ __forceinline__ void check_fail(const flide_tree_index &x, int site, long val) {
+  if (atomicCAS(&x.counts[12], 0, site) == 0) x.counts[13] = (int)val;
+  set_status(x.status, FLIDE_ERR_INVALID);
+}
+
+// 8 bf16 values (one 16-byte chunk q of a 128-byte row) into a swizzled row
+__device__ __forceinline__ void st_chunk(uint8_t *base, int row, int q, uint4 v) {
+  *reinterpret_cast<uint4 *>(base + row * 128 + ((q ^ (row & 7)) << 4)) = v;
+}
+
+// byte offset of element (row, col) in a K-major tile of 128-byte rows
+// (64 bf16 per row) with the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw_elem(int row, int col) {
+  return row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2;
+}
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+  uint4 v;
+  v.x = pack_bf16x2(f[0], f[1]);
+  v.y = pack_bf16x2(f[2], f[3]);
+  v.z = pack_bf16x2(f[4], f[5]);
+  v.w = pack_bf16x2(f[6], f[7]);
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const GdnTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sb = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const flide_tree_index &x = p.x;
+  float *sbeta = reinterpret_cast<float *>(smem + SM_SCAL);
+  float *sG = sbeta + C;
+  float *sgam = sG + C;
+  int *sseg = reinterpret_cast<int *>(sgam + C);
+  float *Am = reinterpret_cast<float *>(smem + SM_A);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
+  int *abort_flag = reinterpret_cast<int *>(smem + SM_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return sb + SM_BAR + 8 * i; };
+
+  if (tid == 0) {
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(bar(i), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tmem_alloc(sb + SM_MISC, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+  volatile int *vabort = abort_flag;
+
+  const int n_groups = failed(x.status) ? 0 : *groups_n(x, p.goff);
+  const int L0 = x.level_ptr[p.level];
+  const long items = (long)n_groups * p.H;
+  uint32_t full_phase0 = 0, full_phase1 = 0, mma_phase = 0;
+  bool pending0 = false, pending1 = false;  // loads in flight (thread 0)
+  int stage = 0;
+  bool ok = true;
+
+  auto mma_sync = [&]() -> bool {  // commit all issued MMAs and wait (every thread)
+    tc_fence_before();
+    if (tid == 0) mma_commit(bar(B_MMA));
+    __syncwarp();
+    const bool r = mbar_wait(bar(B_MMA), mma_phase, vabort, kTimeoutNs);
+    mma_phase ^= 1;
+    tc_fence_after();
+    return __syncthreads_and(r);
+  };
+
+  for (long it = blockIdx.x; ok && it < items; it += gridDim.x) {
+    const int grp = (int)(it / p.H), h = (int)(it % p.H);
+    const int k0 = groups_start(x, p.goff)[grp], cnt = groups_count(x, p.goff)[grp];
+    const int Nact = x.counts[FLIDE_CNT_N], Tact = x.counts[FLIDE_CNT_T];
+    if (k0 < 0 || cnt < 1 || L0 + k0 + cnt > Nact) {
+      if (tid == 0) check_fail(x, 1, k0 * 100000L + cnt);
+      break;
+    }
+    const int n0 = x.level_node[L0 + k0];
+    const int n1 = x.level_node[L0 + k0 + cnt - 1];
+    if (n0 < 0 || n1 < n0 || n1 >= Nact) {
+      if (tid == 0) check_fail(x, 2, n0 * 100000L + n1);
+      break;
+    }
+    const int tbeg = x.node_start[n0], tend = x.node_start[n1 + 1];
+    if (tbeg < 0 || tend < tbeg || tend > Tact) {
+      if (tid == 0) check_fail(x, 3, tend);
+      break;
+    }
+    const bool scan = cnt == 1;  // single node: chunks in order, state carried
+    const int slot = x.state_slot[n0];
+    const int r = x.node_req[n0];
+    if (r < 0 || r >= x.R || (slot >= 0 && slot >= p.n_slots)) {
+      if (tid == 0) check_fail(x, 4, r * 100000L + slot);
+      break;
+    }
+    const int nchunks = (tend - tbeg + C - 1) / C;
+
+    // ---- starting state into TMEM (lane c = state row c)
+    const float *src = nullptr;
+    if (p.level == 0) {
+      if (p.state_in) src = p.state_in + ((size_t)r * p.H + h) * D * D;
+    } else {
+      const int pa = x.anc_ptr[n0 + 1] - 2;
+      const int ps = (pa >= 0 && x.depth[n0] >= 1) ? x.state_slot[x.anc_node[pa]] : -1;
+      if (ps < 0 || ps >= p.n_slots) {
+        if (tid == 0) check_fail(x, 5, ps);
+        break;
+      }
+      src = p.node_state + ((size_t)ps * p.H + h) * D * D;
+    }
+    for (int half = 0; half < 2; ++half) {
+      uint32_t v[64];
+#pragma unroll
+      for (int i = 0; i < 64; i += 4) {
+        const float4 f4 = src ? *reinterpret_cast<const float4 *>(src + (size_t)tid * D + half * 64 + i)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[i] = __float_as_uint(f4.x);
+        v[i + 1] = __float_as_uint(f4.y);
+        v[i + 2] = __float_as_uint(f4.z);
+        v[i + 3] = __float_as_uint(f4.w);
+      }
+      tmem_st64(tl + R_S + half * 64, v);
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // K, Q, V of chunk c into stage st (thread 0)
+    auto issue_loads = [&](int c, int st) {
+      const int row = tbeg + c * C;
+      const uint32_t kq = sb + SM_KQ + st * 32768, vv = sb + SM_V + st * 16384;
+      const uint32_t fb = bar(B_FULL + st);
+      if (st == 0) pending0 = true; else pending1 = true;
+      mbar_arrive_expect_tx(fb, 6 * 8192);
+      tma_load_3d(kq, &tm_k, fb, 0, h, row);
+      tma_load_3d(kq + 16384, &tm_k, fb, 64, h, row);
+      tma_load_3d(kq + 8192, &tm_q, fb, 0, h, row);
+      tma_load_3d(kq + 16384 + 8192, &tm_q, fb, 64, h, row);
+      tma_load_3d(vv, &tm_v, fb, 0, h, row);
+      tma_load_3d(vv + 8192, &tm_v, fb, 64, h, row);
+    };
+    if (tid == 0) issue_loads(0, stage);
+    __syncwarp();
+
+    for (int c = 0; ok && c < nchunks; ++c) {
+      const int st = stage;
+      const int cbeg = tbeg + c * C;
+      const int n = min(C, tend - cbeg);
+      const bool update = scan && (c + 1 < nchunks || slot >= 0);
+      const uint32_t kq = sb + SM_KQ + st * 32768, vv = sb + SM_V + st * 16384;
+      // prefetch the next chunk into the other stage (its last readers are done)
+      if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1, st ^ 1);
+      __syncwarp();
+
+      // ---- per-token scalars: beta, segment id, then the segmented log decay
+      if (tid < C) {
+        const int t = cbeg + tid;
+        const bool v = tid < n && t < Tact;
+        sbeta[tid] = v ? p.beta[(size_t)t * p.H + h] : 0.f;
+        sG[tid] = v ? p.g[(size_t)t * p.H + h] : 0.f;
+        sseg[tid] = v ? x.token_node[t] - n0 : -1;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // segmented inclusive scan of g, two tokens per lane: (value,
+        // segment-start flag) pairs combined Hillis-Steele style
+        const int lane = tid;
+        const float a0 = sG[2 * lane], a1 = sG[2 * lane + 1];
+        const int s0 = sseg[2 * lane], s1 = sseg[2 * lane + 1];
+        const int prev_s1 = __shfl_up_sync(0xffffffffu, s1, 1);
+        const bool cont0 = lane > 0 && prev_s1 == s0;  // token 2l continues token 2l-1
+        float v = (s1 == s0) ? a0 + a1 : a1;
+        int f = (s1 != s0 || !cont0) ? 1 : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float pv = __shfl_up_sync(0xffffffffu, v, o);
+          const int pf = __shfl_up_sync(0xffffffffu, f, o);
+          if (lane >= o) {
+            if (!f) v += pv;
+            f |= pf;
+          }
+        }
+        const float carry = __shfl_up_sync(0xffffffffu, v, 1);
+        const float g0 = a0 + (cont0 ? carry : 0.f);
+        const float g1 = (s1 == s0) ? g0 + a1 : a1;
+        sG[2 * lane] = g0;
+        sG[2 * lane + 1] = g1;
+        sgam[2 * lane] = expf(g0);
+        sgam[2 * lane + 1] = expf(g1);
+      }
+      // ---- wait for this chunk's K, Q, V
+      const bool loaded = mbar_wait(bar(B_FULL + st), st == 0 ? full_phase0 : full_phase1, vabort,
+                                    kTimeoutNs);
+      if (loaded) {
+        if (st == 0) { full_phase0 ^= 1; pending0 = false; }
+        else { full_phase1 ^= 1; pending1 = false; }
+      }
+      if (!__syncthreads_and(loaded)) { ok = false; break; }
+      const float gam_last = sgam[n - 1];
+
+      // ---- R1 = [K;Q] [K;Q]^T
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + R1, sdesc_sw128(kq + o, 16, 1024), sdesc_sw128(kq + o, 16, 1024), id,
+                   kk > 0 ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+      // ---- meanwhile: bf16 copy of S0 (B operand, rows = dv); rescale S
+      {
+        uint32_t sr[128];
+        tmem_ld128(tl + R_S, sr);
+        uint8_t *s0 = smem + SM_S0;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
+          st_chunk(s0 + (q >> 3) * 16384, tid, q & 7, pack8(f));
+        }
+        if (update) {
+          uint32_t a[64], b2[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            a[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
+            b2[i] = __float_as_uint(__uint_as_float(sr[64 + i]) * gam_last);
+          }
+          tmem_st64(tl + R_S, a);
+          tmem_st64(tl + R_S + 64, b2);
+        }
+      }
+      if (!mma_sync()) { ok = false; break; }
+
+      // ---- A (rows 0-63 of R1) and the decayed causal QK^T (rows 64-127)
+      {
+        uint32_t d1[64];
+        tmem_ld32(tl + R1, *reinterpret_cast<uint32_t(*)[32]>(d1));
+        tmem_ld32(tl + R1 + 32, *reinterpret_cast<uint32_t(*)[32]>(d1 + 32));
+        if (tid < C) {
+          const int i = tid;
+          const float bi = sbeta[i], Gi = sG[i];
+          const int si = sseg[i];
+#pragma unroll
+          for (int j = 0; j < C; ++j) {
+            const bool m = j < i && sseg[j] == si && si >= 0;
+            Am[i * A_LD + j] = m ? bi * __expf(Gi - sG[j]) * __uint_as_float(d1[j]) : 0.f;
+          }
+        } else {
+          const int i = tid - C;
+          const float Gi = sG[i];
+          const int si = sseg[i];
+          uint8_t *pm = smem + SM_PM;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float e[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int j = 8 * q + u;
+              const bool m = j <= i && sseg[j] == si && si >= 0;
+              e[u] = m ? __expf(Gi - sG[j]) * __uint_as_float(d1[j]) : 0.f;
+            }
+            st_chunk(pm, tid, q, pack8(e));  // token row i at tile row 64 + i
+          }
+        }
+      }
+      __syncthreads();
+
+      // ---- T = (I + A)^-1, one column per thread; T' and T'' as A operands
+      if (tid < C) {
+        const int col = tid;
+        float tc[C];
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+          const float *arow = Am + i * A_LD;
+#pragma unroll
+          for (int j = 0; j + 3 < i; j += 4) {
+            s0 = fmaf(arow[j], tc[j], s0);
+            s1 = fmaf(arow[j + 1], tc[j + 1], s1);
+            s2 = fmaf(arow[j + 2], tc[j + 2], s2);
+            s3 = fmaf(arow[j + 3], tc[j + 3], s3);
+          }
+#pragma unroll
+          for (int j = i & ~3; j < i; ++j) s0 = fmaf(arow[j], tc[j], s0);
+          const float sum = (s0 + s1) + (s2 + s3);
+          tc[i] = (i == col) ? 1.f : (i > col ? -sum : 0.f);
+        }
+        const float bg = sbeta[col] * sgam[col], bb = sbeta[col];
+        __nv_bfloat16 *t1 = reinterpret_cast<__nv_bfloat16 *>(smem + SM_TA);
+        __nv_bfloat16 *t2 = reinterpret_cast<__nv_bfloat16 *>(smem + SM_TA + 16384);
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+          const uint32_t off = sw_elem(i, col) >> 1;
+          t1[off] = __float2bfloat16_rn(tc[i] * bg);
+          t2[off] = __float2bfloat16_rn(tc[i] * bb);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+
+      // ---- R2 = T' K (= W),  R3 = T'' V (= U)
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_bf16(tmem + R2, sdesc_sw128(sb + SM_TA + kk * 32, 16, 1024),
+                   sdesc_sw128(kq + kk * 2048, 16384, 1024), id, kk > 0 ? 1u : 0u);
+          mma_bf16(tmem + R3, sdesc_sw128(sb + SM_TA + 16384 + kk * 32, 16, 1024),
+                   sdesc_sw128(vv + kk * 2048, 8192, 1024), id, kk > 0 ? 1u : 0u);
+        }
+      }
+      if (!mma_sync()) { ok = false; break; }
+
+      // ---- -W (token rows) as a K-major A operand over T' / T''
+      if (tid < C) {
+        uint32_t w[128];
+        tmem_ld128(tl + R2, w);
+        uint8_t *nw = smem + SM_TA;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(w[8 * q + u]);
+          st_chunk(nw + (q >> 3) * 16384, tid, q & 7, pack8(f));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+
+      // ---- R3 += (-W) S0^T (= Delta);  R1 = [K;Q] S0^T (rows 64-127: Q S0^T)
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint64_t b = sdesc_sw128(sb + SM_S0 + o, 16, 1024);
+          mma_bf16(tmem + R3, sdesc_sw128(sb + SM_TA + o, 16, 1024), b, id, 1u);
+          mma_bf16(tmem + R1, sdesc_sw128(kq + o, 16, 1024), b, id, kk > 0 ? 1u : 0u);
+        }
+      }
+      if (!mma_sync()) { ok = false; break; }
+
+      // ---- Delta rows (token j) -> MN-major B over S0's first half, and
+      //      Delta'^T = (Delta * gamma_last/gamma_j)^T -> K-major A (second half)
+      if (tid < C) {
+        const int j = tid;
+        uint32_t dr[128];
+        tmem_ld128(tl + R3, dr);
+        uint8_t *db = smem + SM_S0;
+        __nv_bfloat16 *dat = reinterpret_cast<__nv_bfloat16 *>(smem + SM_S0 + 16384);
+        const float sc = gam_last / sgam[j];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(dr[8 * q + u]);
+          st_chunk(db + (q >> 3) * 8192, j, q & 7, pack8(f));
+        }
+        if (update) {
+#pragma unroll
+          for (int cdv = 0; cdv < D; ++cdv)
+            dat[sw_elem(cdv, j) >> 1] = __float2bfloat16_rn(__uint_as_float(dr[cdv]) * sc);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+
+      // ---- R2 = (M o QK^T) Delta (rows 64-127);  S += Delta'^T K
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_bf16(tmem + R2, sdesc_sw128(sb + SM_PM + kk * 32, 16, 1024),
+                   sdesc_sw128(sb + SM_S0 + kk * 2048, 8192, 1024), id, kk > 0 ? 1u : 0u);
+          if (update)
+            mma_bf16(tmem + R_S, sdesc_sw128(sb + SM_S0 + 16384 + kk * 32, 16, 1024),
+                     sdesc_sw128(kq + kk * 2048, 16384, 1024), id, 1u);
+        }
+      }
+      if (!mma_sync()) { ok = false; break; }
+
+      // ---- outputs (token rows 64-127): o_i = gamma_i (Q S0^T)_i + ((M o QK^T) Delta)_i
+      if (tid >= C) {
+        const int i = tid - C;
+        const bool valid = i < n && cbeg + i < Tact;
+        __nv_bfloat16 *o = p.out + ((size_t)(cbeg + i) * p.H + h) * D;
+        const float gi = sgam[i];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o1[32], o2[32];
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            tmem_ld32(tl + R1 + half * 64 + qq * 32, o1);
+            tmem_ld32(tl + R2 + half * 64 + qq * 32, o2);
+            if (valid) {
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                float f[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  f[u] = fmaf(gi, __uint_as_float(o1[q8 * 8 + u]), __uint_as_float(o2[q8 * 8 + u]));
+                *reinterpret_cast<uint4 *>(o + half * 64 + qq * 32 + q8 * 8) = pack8(f);
+              }
+            }
+          }
+        }
+      }
+      stage ^= 1;
+      __syncthreads();
+    }
+    if (!ok) break;
+
+    // ---- end state of a node with a slot
+    if (scan && slot >= 0) {
+      uint32_t sr[128];
+      tmem_ld128(tl + R_S, sr);
+      float *dst = p.node_state + ((size_t)slot * p.H + h) * D * D + (size_t)tid * D;
+#pragma unroll
+      for (int i = 0; i < 128; i += 4)
+        *reinterpret_cast<float4 *>(dst + i) =
+            make_float4(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1]),
+                        __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+    }
+    __syncthreads();
+  }
+
+  if (!ok) {
+    // drain: loads this CTA may still have in flight, and its MMAs
+    if (tid == 0) {
+      if (pending0) mbar_wait(bar(B_FULL + 0), full_phase0, vabort, kTimeoutNs, false);
+      if (pending1) mbar_wait(bar(B_FULL + 1), full_phase1, vabort, kTimeoutNs, false);
+      mma_commit(bar(B_MMA));
+      mbar_wait(bar(B_MMA), mma_phase, vabort, kTimeoutNs, false);
+      set_status(x.status, FLIDE_ERR_TIMEOUT);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---- host ------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_gdn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// [rows, heads, 128] bf16 as a 3-D tensor (dim, head, row); box 64 x 1 x 64
+bool make_map_gdn(CUtensorMap *m, const void *base, int heads, long rows) {
+  EncodeTiledFn enc = encode_fn_gdn();
+  if (!enc || rows <= 0) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {256, (cuuint64_t)heads * 256};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)C};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool fork_gdn_tc_supported(int dk, int dv, int dtype) {
+  return dtype == FLIDE_BF16 && dk == D && dv == D && encode_fn_gdn() != nullptr;
+}
+
+int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                const float *state_in, const flide_tree_index *x, int H, void *out,
+                float *node_state, int n_slots, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  const long T = x->T > 0 ? x->T : 1;
+  if (!make_map_gdn(&mq, q, H, T) || !make_map_gdn(&mk, k, H, T) || !make_map_gdn(&mv, v, H, T))
+    return FLIDE_ERR_CUDA;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLIDE_ERR_CUDA;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    if (cudaFuncSetAttribute(gdn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return FLIDE_ERR_CUDA;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  GdnTcParams prm;
+  prm.x = *x;
+  prm.g = g;
+  prm.beta = beta;
+  prm.state_in = state_in;
+  prm.out = (__nv_bfloat16 *)out;
+  prm.node_state = node_state;
+  prm.H = H;
+  prm.n_slots = n_slots;
+  prm.goff = 4 * (x->R + 1);  // after the attention's per-request table
+  for (int lvl = 0; lvl <= x->max_depth; ++lvl) {
+    prm.level = lvl;
+    gdn_groups_kernel<<<1, 1024, 0, s>>>(*x, lvl, prm.goff);
+    FLIDE_LAUNCH_CHECK();
+    gdn_tc_kernel<<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
+    FLIDE_LAUNCH_CHECK();
+  }
+  return FLIDE_OK;
+}
+
+}  // namespace flide

@@ -205,5 +205,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::f16 with every option: fp32 accumulator,
+// bf16 A and B, A/B K-major (false) or MN-major (true), optional negation of A.
+__host__ __device__ constexpr uint32_t idesc_bf16_ex(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                     bool negate_a) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((negate_a ? 1u : 0u) << 13) |
+         ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 }  // namespace sm100
 }  // namespace flide
