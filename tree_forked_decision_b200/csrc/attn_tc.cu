@@ -399,9 +399,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tile_at(ms, j, sp, off);
         uint32_t sr[128];
         tmem_ld128(t_s, sr);
-        float sv[128];
-#pragma unroll
-        for (int i = 0; i < 128; ++i) sv[i] = __uint_as_float(sr[i]);
         const int rem = sp.len - off;
         if (sp.kind != KIND_FULL || rem < BN) {
           const int key0 = sp.start + off;
@@ -417,16 +414,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               const int kn = vis ? x.token_node[key] : -1;
               vis = vis && kn == a_row && (kn != row_node || key <= t);
             }
-            if (!vis) sv[i] = -INFINITY;
+            if (!vis) sr[i] = 0xff800000u;  // -inf
           }
         }
+        // row max: 8 chains of three-input max
         float mx[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
 #pragma unroll
-        for (int i = 8; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
-        const float smax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int i = 8; i < BN; i += 16) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx[k] = fmax3f(mx[k], __uint_as_float(sr[i + 2 * k]), __uint_as_float(sr[i + 2 * k + 1]));
+        }
+        const float smax = fmaxf(fmax3f(mx[0], mx[1], mx[2]),
+                                 fmax3f(fmax3f(mx[3], mx[4], mx[5]), mx[6], mx[7]));
         const float mt = smax * c;
         if (j == 0) {
           m_used = mt;
@@ -448,19 +450,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
         }
         const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-        float ps[8];
+        // p = 2^(s*c - m): paired scale-and-shift, SFU exp2, paired row-sum
+        // chains; P packed to bf16x2 in place into sr[0..63]
+        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_sub, -m_sub);
+        uint64_t acc[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ps[i] = 0.f;
-        uint32_t pk[64];
+        for (int k = 0; k < 4; ++k) acc[k] = 0ull;
 #pragma unroll
         for (int i = 0; i < BN; i += 2) {
-          const float e0 = ex2_approx(fmaf(sv[i], c, -m_sub));
-          const float e1 = ex2_approx(fmaf(sv[i + 1], c, -m_sub));
-          ps[(i >> 1) & 7] += e0 + e1;
-          pk[i >> 1] = pack_bf16x2(e0, e1);
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2), x0, x1);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          acc[(i >> 1) & 3] = f2_add(acc[(i >> 1) & 3], f2_pack(e0, e1));
+          sr[i >> 1] = pack_bf16x2(e0, e1);
         }
-        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        tmem_st64(t_s, pk);
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2_unpack(acc[0], a0, a1);
+          f2_unpack(acc[1], b0, b1);
+          f2_unpack(acc[2], c0, c1);
+          f2_unpack(acc[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
+        tmem_st64(t_s, *reinterpret_cast<uint32_t(*)[64]>(sr));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_FULL + h));
