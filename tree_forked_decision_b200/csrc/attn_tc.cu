@@ -387,6 +387,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const uint32_t t_s = tl + h * 256, t_o = tl + h * 256 + 128;
       const float c = p.qk_log2;
       float m_used = -INFINITY, l = 0.f;
+      int span_tile0 = -1, vis_lo = 0, vis_hi = 0;
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + h), j & 1, abort_flag, kTimeoutNs))) {
@@ -399,22 +400,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tile_at(ms, j, sp, off);
         uint32_t sr[128];
         tmem_ld128(t_s, sr);
-        const int rem = sp.len - off;
-        if (sp.kind != KIND_FULL || rem < BN) {
-          const int key0 = sp.start + off;
-          const int a_row = (sp.kind == KIND_TREE && valid_row && row_depth >= sp.level)
-                                ? x.anc_node[row_anc + sp.level]
-                                : -2;
-#pragma unroll
-          for (int i = 0; i < BN; ++i) {
-            bool vis = i < rem;
-            const int key = key0 + i;
-            if (sp.kind == KIND_CAUSAL) vis = vis && key <= t;
-            if (sp.kind == KIND_TREE) {
-              const int kn = vis ? x.token_node[key] : -1;
-              vis = vis && kn == a_row && (kn != row_node || key <= t);
+        // The keys this row sees inside one span form one range [vis_lo,
+        // vis_hi) of key indices: the whole span (past rows, the root for a
+        // branch tile), keys up to the row's own token (causal root), or the
+        // token segment of the row's level-L ancestor, cut after the row's
+        // own token when that ancestor is the row's own node (tree level).
+        // The range is refreshed when the span changes; a tile is masked
+        // with two integer bounds, and not at all when it is fully visible
+        // to every row of the warp.
+        if (sp.tile0 != span_tile0) {
+          span_tile0 = sp.tile0;
+          vis_lo = sp.start;
+          vis_hi = sp.start + sp.len;
+          if (valid_row && sp.kind == KIND_CAUSAL) {
+            vis_hi = min(vis_hi, t + 1);
+          } else if (valid_row && sp.kind == KIND_TREE) {
+            if (row_depth >= sp.level) {
+              const int a = x.anc_node[row_anc + sp.level];
+              vis_lo = x.node_start[a];
+              vis_hi = a == row_node ? t + 1 : x.node_start[a + 1];
+            } else {
+              vis_hi = vis_lo;
             }
-            if (!vis) sr[i] = 0xff800000u;  // -inf
+          }
+          vis_hi = max(vis_hi, vis_lo);
+        }
+        {
+          const int key0 = sp.start + off;
+          const int lo = min(max(vis_lo - key0, 0), BN), hi = min(max(vis_hi - key0, 0), BN);
+          if (!__all_sync(0xffffffffu, lo == 0 && hi == BN)) {
+            const uint32_t w = (uint32_t)(hi - lo);
+#pragma unroll
+            for (int i = 0; i < BN; ++i)
+              if ((uint32_t)(i - lo) >= w) sr[i] = 0xff800000u;  // -inf
           }
         }
         // row max: 8 chains of three-input max
