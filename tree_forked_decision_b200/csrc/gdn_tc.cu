@@ -22,7 +22,9 @@
 //   R2 = T' K,  R3 = T'' V -> W and U (T' = T diag(b gamma), T'' = T diag(b))
 //   R3 += (-W) S0^T        -> Delta         R1 = [K;Q] S0^T -> Q S0^T (rows 64-127)
 //   R2 = (M o QK^T) Delta  -> rows 64-127   S += Delta'^T K  (Delta' = Delta gamma_last/gamma)
-// T is solved in fp32 on CUDA cores (one column per thread).  The fp32 state
+// T is solved in fp32 on CUDA cores by 16 x 16 blocks: the four diagonal
+// blocks by substitution, then block row i from T_ij = -T_ii sum_k A_ik T_kj.
+// The fp32 state
 // lives in TMEM for the whole scan; a bf16 copy is the operand for a chunk.
 //
 // Work items (built per level by gdn_groups_kernel): a root, an inner node or
@@ -57,8 +59,11 @@ constexpr int SM_TA = 131072;   // T' and T'' [128 rows][64] K-major (16 KB each
 constexpr int SM_PM = 163840;   // (M o QK^T) [128 rows][64] K-major, token rows at 64-127
 constexpr int SM_A = 180224;    // fp32 A [64][65]
 constexpr int A_LD = 65;
-constexpr int SM_SCAL = SM_A + C * A_LD * 4;  // beta, G, gamma, seg: 4 x 64 words
-constexpr int SM_BAR = SM_SCAL + 4 * C * 4;
+constexpr int SM_T = SM_A + C * A_LD * 4;     // fp32 T [64][65]
+constexpr int SM_X = SM_T + C * A_LD * 4;     // fp32 block products X [3][16][17]
+constexpr int X_LD = 17;
+constexpr int SM_SCAL = SM_X + 3 * 16 * X_LD * 4;  // beta, G, gamma, seg, G*log2(e): 5 x 64 words
+constexpr int SM_BAR = SM_SCAL + 5 * C * 4;
 constexpr int SM_MISC = SM_BAR + 64;
 constexpr int SMEM_BYTES = SM_MISC + 64 + 1024;
 
@@ -182,6 +187,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   float *sG = sbeta + C;
   float *sgam = sG + C;
   int *sseg = reinterpret_cast<int *>(sgam + C);
+  float *sG2 = reinterpret_cast<float *>(sseg + C);  // G * log2(e)
   float *Am = reinterpret_cast<float *>(smem + SM_A);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
   int *abort_flag = reinterpret_cast<int *>(smem + SM_MISC + 4);
@@ -295,6 +301,18 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     };
     if (tid == 0) issue_loads(0, stage);
     __syncwarp();
+    // per-token scalars (beta, g, node) of the next chunk, loaded into
+    // registers one chunk ahead so their latency overlaps the current chunk
+    float nb = 0.f, ng = 0.f;
+    int nn = -1;
+    auto load_scalars = [&](int c) {
+      const int t = tbeg + c * C + tid;
+      const bool v = tid < C && t < tend && t < Tact;
+      nb = v ? p.beta[(size_t)t * p.H + h] : 0.f;
+      ng = v ? p.g[(size_t)t * p.H + h] : 0.f;
+      nn = v ? x.token_node[t] - n0 : -1;
+    };
+    load_scalars(0);
 
     for (int c = 0; ok && c < nchunks; ++c) {
       const int st = stage;
@@ -308,12 +326,11 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
       // ---- per-token scalars: beta, segment id, then the segmented log decay
       if (tid < C) {
-        const int t = cbeg + tid;
-        const bool v = tid < n && t < Tact;
-        sbeta[tid] = v ? p.beta[(size_t)t * p.H + h] : 0.f;
-        sG[tid] = v ? p.g[(size_t)t * p.H + h] : 0.f;
-        sseg[tid] = v ? x.token_node[t] - n0 : -1;
+        sbeta[tid] = nb;
+        sG[tid] = ng;
+        sseg[tid] = nn;
       }
+      if (c + 1 < nchunks) load_scalars(c + 1);
       __syncthreads();
       if (warp == 0) {
         // segmented inclusive scan of g, two tokens per lane: (value,
@@ -341,6 +358,8 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         sG[2 * lane + 1] = g1;
         sgam[2 * lane] = expf(g0);
         sgam[2 * lane + 1] = expf(g1);
+        sG2[2 * lane] = g0 * 1.4426950408889634f;
+        sG2[2 * lane + 1] = g1 * 1.4426950408889634f;
       }
       // ---- wait for this chunk's K, Q, V
       const bool loaded = mbar_wait(bar(B_FULL + st), st == 0 ? full_phase0 : full_phase1, vabort,
@@ -389,68 +408,146 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       if (!mma_sync()) { ok = false; break; }
 
-      // ---- A (rows 0-63 of R1) and the decayed causal QK^T (rows 64-127)
+      // ---- A (rows 0-63 of R1) and the decayed causal QK^T (rows 64-127):
+      //      entry (i, j) scaled by gamma_i / gamma_j = 2^(G2_i - G2_j) where
+      //      j precedes (A) or equals (QK^T) i inside i's segment
       {
         uint32_t d1[64];
         tmem_ld32(tl + R1, *reinterpret_cast<uint32_t(*)[32]>(d1));
         tmem_ld32(tl + R1 + 32, *reinterpret_cast<uint32_t(*)[32]>(d1 + 32));
-        if (tid < C) {
-          const int i = tid;
-          const float bi = sbeta[i], Gi = sG[i];
-          const int si = sseg[i];
+        const int i = tid & (C - 1);
+        const bool is_a = tid < C;
+        const float G2i = sG2[i], scale_i = is_a ? sbeta[i] : 1.f;
+        const int si = sseg[i];
+        const int jmax = is_a ? i - 1 : i;  // last visible j
+        const float4 *g4 = reinterpret_cast<const float4 *>(sG2);
+        const int4 *s4 = reinterpret_cast<const int4 *>(sseg);
+        float e[64];
 #pragma unroll
-          for (int j = 0; j < C; ++j) {
-            const bool m = j < i && sseg[j] == si && si >= 0;
-            Am[i * A_LD + j] = m ? bi * __expf(Gi - sG[j]) * __uint_as_float(d1[j]) : 0.f;
+        for (int q = 0; q < 16; ++q) {
+          const float4 gv = g4[q];
+          const int4 sv = s4[q];
+          const float gj[4] = {gv.x, gv.y, gv.z, gv.w};
+          const int sj[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = 4 * q + u;
+            const bool m = j <= jmax && sj[u] == si && si >= 0;
+            e[j] = m ? scale_i * ex2_approx(G2i - gj[u]) * __uint_as_float(d1[j]) : 0.f;
           }
+        }
+        if (is_a) {
+#pragma unroll
+          for (int j = 0; j < C; ++j) Am[i * A_LD + j] = e[j];
         } else {
-          const int i = tid - C;
-          const float Gi = sG[i];
-          const int si = sseg[i];
           uint8_t *pm = smem + SM_PM;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float e[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int j = 8 * q + u;
-              const bool m = j <= i && sseg[j] == si && si >= 0;
-              e[u] = m ? __expf(Gi - sG[j]) * __uint_as_float(d1[j]) : 0.f;
-            }
-            st_chunk(pm, tid, q, pack8(e));  // token row i at tile row 64 + i
-          }
+          for (int q = 0; q < 8; ++q) st_chunk(pm, tid, q, pack8(e + 8 * q));  // token row i at tile row 64 + i
         }
       }
       __syncthreads();
 
-      // ---- T = (I + A)^-1, one column per thread; T' and T'' as A operands
-      if (tid < C) {
-        const int col = tid;
-        float tc[C];
+      // ---- T = (I + A)^-1 by 16 x 16 blocks (A strictly lower triangular)
+      {
+        float *Tm = reinterpret_cast<float *>(smem + SM_T);
+        float *Xm = reinterpret_cast<float *>(smem + SM_X);
+        // diagonal blocks: thread (block kb, column cc), substitution down the column
+        if (tid < C) {
+          const int r0 = 16 * (tid >> 4), cc = tid & 15;
+          float tcol[16];
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-          const float *arow = Am + i * A_LD;
+          for (int i = 0; i < 16; ++i) {
+            float s0 = 0.f, s1 = 0.f;
+            const float *arow = Am + (r0 + i) * A_LD + r0;
 #pragma unroll
-          for (int j = 0; j + 3 < i; j += 4) {
-            s0 = fmaf(arow[j], tc[j], s0);
-            s1 = fmaf(arow[j + 1], tc[j + 1], s1);
-            s2 = fmaf(arow[j + 2], tc[j + 2], s2);
-            s3 = fmaf(arow[j + 3], tc[j + 3], s3);
+            for (int j = 0; j + 1 < i; j += 2) {
+              s0 = fmaf(arow[j], tcol[j], s0);
+              s1 = fmaf(arow[j + 1], tcol[j + 1], s1);
+            }
+            if (i & 1) s0 = fmaf(arow[i - 1], tcol[i - 1], s0);
+            tcol[i] = (i == cc) ? 1.f : (i > cc ? -(s0 + s1) : 0.f);
           }
 #pragma unroll
-          for (int j = i & ~3; j < i; ++j) s0 = fmaf(arow[j], tc[j], s0);
-          const float sum = (s0 + s1) + (s2 + s3);
-          tc[i] = (i == col) ? 1.f : (i > col ? -sum : 0.f);
+          for (int i = 0; i < 16; ++i) Tm[(r0 + i) * A_LD + r0 + cc] = tcol[i];
         }
-        const float bg = sbeta[col] * sgam[col], bb = sbeta[col];
-        __nv_bfloat16 *t1 = reinterpret_cast<__nv_bfloat16 *>(smem + SM_TA);
-        __nv_bfloat16 *t2 = reinterpret_cast<__nv_bfloat16 *>(smem + SM_TA + 16384);
+        __syncthreads();
+        // block row bi: X_bj = sum_{k=j}^{bi-1} A_bk T_kj, then T_bj = -T_bb X_bj.
+        // Thread -> (row r of the block row, column pair 2cp, 2cp+1) for every
+        // column block j < bi: up to six independent sums, each A value
+        // loaded once for two columns.
+        {
+          const int r = tid >> 3, cp = tid & 7;
+          for (int bi = 1; bi < 4; ++bi) {
+            const float *arow = Am + (16 * bi + r) * A_LD;
+            float acc[3][2];
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-          const uint32_t off = sw_elem(i, col) >> 1;
-          t1[off] = __float2bfloat16_rn(tc[i] * bg);
-          t2[off] = __float2bfloat16_rn(tc[i] * bb);
+            for (int jb = 0; jb < 3; ++jb) acc[jb][0] = acc[jb][1] = 0.f;
+#pragma unroll
+            for (int kb = 0; kb < 3; ++kb) {
+              if (kb >= bi) break;
+#pragma unroll
+              for (int m = 0; m < 16; ++m) {
+                const float a = arow[16 * kb + m];
+                const float *trow = Tm + (16 * kb + m) * A_LD + 2 * cp;
+#pragma unroll
+                for (int jb = 0; jb < 3; ++jb) {
+                  if (jb <= kb) {
+                    acc[jb][0] = fmaf(a, trow[16 * jb], acc[jb][0]);
+                    acc[jb][1] = fmaf(a, trow[16 * jb + 1], acc[jb][1]);
+                  }
+                }
+              }
+            }
+#pragma unroll
+            for (int jb = 0; jb < 3; ++jb) {
+              if (jb < bi) {
+                Xm[(jb * 16 + r) * X_LD + 2 * cp] = acc[jb][0];
+                Xm[(jb * 16 + r) * X_LD + 2 * cp + 1] = acc[jb][1];
+              }
+            }
+            __syncthreads();
+            const float *trow = Tm + (16 * bi + r) * A_LD + 16 * bi;
+#pragma unroll
+            for (int jb = 0; jb < 3; ++jb) acc[jb][0] = acc[jb][1] = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              const float tv = m <= r ? trow[m] : 0.f;
+#pragma unroll
+              for (int jb = 0; jb < 3; ++jb) {
+                if (jb < bi) {
+                  acc[jb][0] = fmaf(tv, Xm[(jb * 16 + m) * X_LD + 2 * cp], acc[jb][0]);
+                  acc[jb][1] = fmaf(tv, Xm[(jb * 16 + m) * X_LD + 2 * cp + 1], acc[jb][1]);
+                }
+              }
+            }
+#pragma unroll
+            for (int jb = 0; jb < 3; ++jb) {
+              if (jb < bi) {
+                Tm[(16 * bi + r) * A_LD + 16 * jb + 2 * cp] = -acc[jb][0];
+                Tm[(16 * bi + r) * A_LD + 16 * jb + 2 * cp + 1] = -acc[jb][1];
+              }
+            }
+            __syncthreads();
+          }
+        }
+        // T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles:
+        // thread -> (row i, half of the columns)
+        {
+          const int i = tid >> 1, hh = tid & 1;
+          uint8_t *t1 = smem + SM_TA, *t2 = smem + SM_TA + 16384;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float f1[8], f2[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int j = 32 * hh + 8 * q + u;
+              const float tv = (j >> 4) <= (i >> 4) ? Tm[i * A_LD + j] : 0.f;
+              f1[u] = tv * sbeta[j] * sgam[j];
+              f2[u] = tv * sbeta[j];
+            }
+            st_chunk(t1, i, 4 * hh + q, pack8(f1));
+            st_chunk(t2, i, 4 * hh + q, pack8(f2));
+          }
         }
       }
       fence_proxy_async_smem();
