@@ -288,6 +288,27 @@ def dist_env():
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def rank_seed(workload: str, seed, rank: int) -> int:
+    """Seed of this rank's batch: ranks serve independent requests (weak
+    scaling, no data-path collective), so each draws its own inputs."""
+    base = seed if seed is not None else inputs.WORKLOADS[workload]["idx"]
+    return base + 1000 * rank
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    """The job's time is its slowest rank's (a MAX all-reduce)."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return units_per_rank * steps * world / (ms_max / 1000.0)
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -355,8 +376,7 @@ def main():
         pg = dist
     flide.load()
 
-    spec = inputs.WORKLOADS[args.workload]
-    seed = (args.seed if args.seed is not None else spec["idx"]) + 1000 * rank
+    seed = rank_seed(args.workload, args.seed, rank)
     tree, a, g, dtype = inputs.make_inputs(args.workload, seed=seed)
     if args.layers == "attn":
         g = None
@@ -397,12 +417,8 @@ def main():
     gdn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     if step.idx.status() != 0:
         raise SystemExit(f"device status {step.idx.status()} in the timed region")
-    if pg is not None:
-        t = torch.tensor([ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
-    units = tree.branch_tokens * args.steps * ws
-    value = units / (ms / 1000.0)
+    ms = max_over_ranks(ms, pg, device)
+    value = job_throughput(tree.branch_tokens, args.steps, ws, ms)
 
     # end to end through the public API with host buffers: H2D of every input
     # from pinned memory, the call sequence, D2H of every branch token's output
@@ -463,14 +479,10 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        ems = e0.elapsed_time(e1)
-        if pg is not None:
-            t = torch.tensor([ems], device=device)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), pg, device)
         if int(status_h.item()) != 0:
             raise SystemExit(f"device status {int(status_h.item())} in the e2e leg")
-        e2e = {"value": tree.branch_tokens * n_e2e * ws / (ems / 1000.0), "unit": UNIT,
+        e2e = {"value": job_throughput(tree.branch_tokens, n_e2e, ws, ems), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e, "ms_per_step": ems / n_e2e}
 
@@ -484,9 +496,9 @@ def main():
         kernels["fork_gdn"] = {"ms": gdn_ms, "algorithmic_bytes": gbytes, "gbs": gdn_gbs,
                                "frac_of_hbm_peak": gdn_gbs / hbm, "bound": "hbm"}
         roofline = {
-            "kernel": "gdn_level_kernel (GDN fork scan)", "bound": "hbm", "achieved": gdn_gbs,
+            "kernel": "gdn_tc_kernel (GDN fork scan, tcgen05)", "bound": "hbm", "achieved": gdn_gbs,
             "peak": hbm, "unit": "GB/s", "frac": gdn_gbs / hbm,
-            "traffic": traffic_for("gdn_level_kernel", "gdn_portable.cu"),
+            "traffic": traffic_for("gdn_tc_kernel", "gdn_tc.cu"),
             "peak_source": f"{peak_src}: HBM copy bandwidth",
             "algorithmic_bytes_per_launch": gbytes, "avg_launch_ms": gdn_ms}
     if a is not None:
