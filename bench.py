@@ -69,12 +69,19 @@ def attn_work(tree, a):
 
 
 def gdn_work(tree, g, slots):
-    """Algorithmic bytes of one GDN fork scan: q, k, v, out, g, beta once, plus
-    one fp32 state write per saved node and one read per child / resumed root."""
+    """Algorithmic bytes of one GDN fork scan: q, k, v, out, g, beta once, one
+    fp32 state write per saved node, and one state read per parent with
+    children (its checkpoint is broadcast to all its branches) and per resumed
+    root."""
     H, dk, dv = g["H"], g["dk"], g["dv"]
     es = 2 if g["q"].dtype == torch.bfloat16 else 4
     state = 4 * H * dk * dv
-    reads = int(tree.N - tree.R) + int(np.sum(tree.past_len > 0))
+    has_child = np.zeros(tree.N, bool)
+    for r in range(tree.R):
+        for n in range(tree.req_node_ptr[r], tree.req_node_ptr[r + 1]):
+            if tree.parent[n] >= 0:
+                has_child[tree.req_node_ptr[r] + tree.parent[n]] = True
+    reads = int(has_child.sum()) + int(np.sum(tree.past_len > 0))
     byts = tree.T * H * ((2 * dk + 2 * dv) * es + 8) + state * (slots + reads)
     return byts
 
