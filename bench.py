@@ -232,32 +232,37 @@ def cpu_oracle_rate(tree, a, g, attn_rows: int, gdn_pairs: int, seed: int = 0):
 
     rng = np.random.default_rng(seed)
     f32 = lambda t: t.float().numpy()
-    T, Hq = tree.T, a["Hq"]
-    n_rows = T * Hq
-    pick = rng.choice(n_rows, size=min(attn_rows, n_rows), replace=False)
-    rows = np.stack([pick // Hq, pick % Hq], 1).astype(np.int32)
-    qa, ka, va, pka, pva = f32(a["q"]), f32(a["k"]), f32(a["v"]), f32(a["past_k"]), f32(a["past_v"])
-    t0 = time.perf_counter()
-    oracle.attention_rows(tree.arrays(), qa, ka, va, pka, pva, 1.0 / math.sqrt(a["d"]), rows)
-    t_attn = (time.perf_counter() - t0) * n_rows / len(rows)
-    del qa, ka, va
-    H = g["H"]
-    all_pairs = [(r, h) for r in range(tree.R) for h in range(H)]
-    sel = rng.choice(len(all_pairs), size=min(gdn_pairs, len(all_pairs)), replace=False)
-    heads = sorted({all_pairs[i][1] for i in sel})
-    # slice the selected heads so the oracle reads only their data
-    hq = lambda t: np.ascontiguousarray(f32(t)[:, heads])
-    pairs = [(all_pairs[i][0], heads.index(all_pairs[i][1])) for i in sel]
-    st = f32(g["state_in"])[:, heads] if np.any(tree.past_len > 0) else None
-    gq, gk, gv, gg, gb = hq(g["q"]), hq(g["k"]), hq(g["v"]), hq(g["g"]), hq(g["beta"])
-    t0 = time.perf_counter()
-    oracle.gdn(tree.arrays(), gq, gk, gv, gg, gb, state_in=st, memoise=True, pairs=pairs)
-    t_gdn = (time.perf_counter() - t0) * len(all_pairs) / len(sel)
+    t_attn = t_gdn = 0.0
+    parts = []
+    if a is not None:
+        T, Hq = tree.T, a["Hq"]
+        n_rows = T * Hq
+        pick = rng.choice(n_rows, size=min(attn_rows, n_rows), replace=False)
+        rows = np.stack([pick // Hq, pick % Hq], 1).astype(np.int32)
+        qa, ka, va = f32(a["q"]), f32(a["k"]), f32(a["v"])
+        pka, pva = f32(a["past_k"]), f32(a["past_v"])
+        t0 = time.perf_counter()
+        oracle.attention_rows(tree.arrays(), qa, ka, va, pka, pva, 1.0 / math.sqrt(a["d"]), rows)
+        t_attn = (time.perf_counter() - t0) * n_rows / len(rows)
+        del qa, ka, va
+        parts.append(f"{len(rows)} of {n_rows} attention query rows")
+    if g is not None:
+        H = g["H"]
+        all_pairs = [(r, h) for r in range(tree.R) for h in range(H)]
+        sel = rng.choice(len(all_pairs), size=min(gdn_pairs, len(all_pairs)), replace=False)
+        heads = sorted({all_pairs[i][1] for i in sel})
+        # slice the selected heads so the oracle reads only their data
+        hq = lambda t: np.ascontiguousarray(f32(t)[:, heads])
+        pairs = [(all_pairs[i][0], heads.index(all_pairs[i][1])) for i in sel]
+        st = f32(g["state_in"])[:, heads] if np.any(tree.past_len > 0) else None
+        gq, gk, gv, gg, gb = hq(g["q"]), hq(g["k"]), hq(g["v"]), hq(g["g"]), hq(g["beta"])
+        t0 = time.perf_counter()
+        oracle.gdn(tree.arrays(), gq, gk, gv, gg, gb, state_in=st, memoise=True, pairs=pairs)
+        t_gdn = (time.perf_counter() - t0) * len(all_pairs) / len(sel)
+        parts.append(f"{len(sel)} of {len(all_pairs)} GDN (request, head) pairs (memoised oracle)")
     rate = tree.branch_tokens / (t_attn + t_gdn)
-    desc = (f"{len(rows)} of {n_rows} attention query rows and {len(sel)} of {len(all_pairs)} "
-            f"GDN (request, head) pairs (memoised oracle), seeded uniform sample; each time "
-            f"scaled by all/sampled units: attention {t_attn:.1f} s + GDN {t_gdn:.1f} s "
-            f"per step extrapolated")
+    desc = (" and ".join(parts) + f", seeded uniform sample; each time scaled by all/sampled "
+            f"units: attention {t_attn:.1f} s + GDN {t_gdn:.1f} s per step extrapolated")
     return rate, desc, oracle.num_threads()
 
 
@@ -525,7 +530,7 @@ def main():
             }
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline and a is not None and g is not None:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, desc, threads = cpu_oracle_rate(tree, a, g, args.cpu_rows, args.cpu_pairs)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
