@@ -134,7 +134,8 @@ class Step:
         self.node_state = torch.empty((self.slots, g["H"], g["dv"], g["dk"]), dtype=torch.float32,
                                       device=device)
         self.cS = torch.empty((tree.R, g["H"], g["dv"], g["dk"]), dtype=torch.float32, device=device)
-        self.launches += (self.dt.max_depth + 1) + 1
+        # per tree level a grouping and a scan launch, then the state save
+        self.launches += 2 * (self.dt.max_depth + 1) + 1
 
     def run(self, ev=None):
         """tree build -> fork attention -> GDN fork scan -> checkpoint save;
@@ -316,6 +317,13 @@ def max_over_ranks(x: float, pg, device) -> float:
     return float(t.item())
 
 
+def percentiles(xs):
+    """(P50, P95) of a list of per-step times (nearest rank)."""
+    v = sorted(xs)
+    pick = lambda q: v[min(len(v) - 1, max(0, int(math.ceil(q * len(v))) - 1))]
+    return pick(0.50), pick(0.95)
+
+
 def job_throughput(units_per_rank: int, steps: int, world: int, ms_max: float) -> float:
     """Whole-job units per second: every rank's units over the slowest rank's time."""
     return units_per_rank * steps * world / (ms_max / 1000.0)
@@ -365,6 +373,8 @@ def main():
                     help="profiling aid: run one layer only (not a headline number)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--no-warm", action="store_true", help="skip the resumed-prefix (warm) timing")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--cpu-pairs", type=int, default=16)
     ap.add_argument("--ref-rows", type=int, default=2000)
@@ -414,23 +424,93 @@ def main():
         raise SystemExit(f"device status {step.idx.status()} after warm-up")
 
     # timed region: inputs resident in HBM (GBs per step, far above the 126 MB L2)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     with ClockSampler(local_rank) as clk:
         start.record()
         for i in range(args.steps):
+            evs[i][3].record()
             step.run(evs[i])
+            evs[i][4].record()
         stop.record()
         torch.cuda.synchronize()
     barrier()
     ms = start.elapsed_time(stop)
     attn_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     gdn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    p50_ms, p95_ms = percentiles([e[3].elapsed_time(e[4]) for e in evs])
+    p50_ms, p95_ms = max_over_ranks(p50_ms, pg, device), max_over_ranks(p95_ms, pg, device)
     if step.idx.status() != 0:
         raise SystemExit(f"device status {step.idx.status()} in the timed region")
     ms = max_over_ranks(ms, pg, device)
     value = job_throughput(tree.branch_tokens, args.steps, ws, ms)
+
+    # the same call sequence captured once as a CUDA graph and replayed
+    graph = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(device=device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step.run()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg):
+            step.run()
+        torch.cuda.synchronize()
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            gev[i][0].record()
+            cg.replay()
+            gev[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        if step.idx.status() != 0:
+            raise SystemExit(f"device status {step.idx.status()} in the graph replays")
+        g50, g95 = percentiles([e[0].elapsed_time(e[1]) for e in gev])
+        g50, g95 = max_over_ranks(g50, pg, device), max_over_ranks(g95, pg, device)
+        graph = {"replays": args.steps, "p50_ms": g50, "p95_ms": g95,
+                 "value_at_p50": job_throughput(tree.branch_tokens, 1, ws, g50), "unit": UNIT}
+        del cg
+
+    # warm: the same batch resumed from this step's checkpoint (past K/V rows
+    # and the roots' end states), so only branch tokens are computed
+    warm = None
+    if not args.no_warm and tree.root_tokens > 0:
+        tree_w, keep = inputs.warm_variant(tree)
+        ridx = torch.from_numpy(keep)
+        a_w = g_w = None
+        if a is not None:
+            a_w = dict(a, q=a["q"][ridx], k=a["k"][ridx], v=a["v"][ridx],
+                       past_k=step.ck[:tree_w.P_past], past_v=step.cv[:tree_w.P_past])
+        if g is not None:
+            g_w = dict(g, state_in=step.cS, **{nm: g[nm][ridx] for nm in ("q", "k", "v", "g", "beta")})
+        wstep = Step(tree_w, a_w, g_w, device)
+        for _ in range(max(args.warmup, 0)):
+            wstep.run()
+        wev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            wev[i][3].record()
+            wstep.run(wev[i])
+            wev[i][4].record()
+        torch.cuda.synchronize()
+        barrier()
+        if wstep.idx.status() != 0:
+            raise SystemExit(f"device status {wstep.idx.status()} in the warm leg")
+        w_steps = [e[3].elapsed_time(e[4]) for e in wev]
+        w_ms = max_over_ranks(statistics.mean(w_steps), pg, device)
+        w50, w95 = percentiles(w_steps)
+        warm = {"value": job_throughput(tree_w.branch_tokens, 1, ws, w_ms), "unit": UNIT,
+                "ms_per_step": w_ms, "p50_ms": max_over_ranks(w50, pg, device),
+                "p95_ms": max_over_ranks(w95, pg, device),
+                "attn_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in wev) if a is not None else None,
+                "gdn_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in wev) if g is not None else None,
+                "resumed_past_rows": tree_w.P_past, "stream_tokens": tree_w.T,
+                "note": "prefix resumed from the timed step's checkpoint; branch tokens only"}
+        del wstep
 
     # end to end through the public API with host buffers: H2D of every input
     # from pinned memory, the call sequence, D2H of every branch token's output
@@ -549,6 +629,9 @@ def main():
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "p50_ms": p50_ms, "p95_ms": p95_ms,
+        "graph": graph,
+        "warm": warm,
         "gpu_launches": step.launches * args.steps,
         "clocks": clk.summary(),
     }

@@ -75,3 +75,5 @@ def test_rank_seed_and_throughput_single_rank():
     assert bench.rank_seed(WORKLOAD, 7, 3) == 3007
     assert bench.max_over_ranks(4.25, None, "cpu") == 4.25
     assert bench.job_throughput(100, 2, 1, 50.0) == 4000.0
+    assert bench.percentiles([5.0, 1.0, 2.0, 3.0, 4.0, 6.0, 7.0, 8.0, 9.0, 10.0]) == (5.0, 10.0)
+    assert bench.percentiles([2.5]) == (2.5, 2.5)

@@ -32,7 +32,8 @@
 // carried in TMEM, end state saved when the node has a slot); runs of
 // consecutive sibling leaves that fit one chunk are packed into one item with
 // a block-diagonal mask, so no leaf sees another.  Items x heads are spread
-// over a persistent grid of one CTA per SM.  Every wait is bounded (2 s).
+// over a persistent grid of one CTA per SM that takes them, longest group
+// first, from a shared counter.  Every wait is bounded (2 s).
 #include <cstddef>
 
 #include "common.cuh"
@@ -81,7 +82,8 @@ struct GdnTcParams {
 };
 
 // work[goff] = number of groups; work[goff+1+g] = first level position of
-// group g; work[goff+2+N+g] = its node count.
+// group g; work[goff+2+N+g] = its node count; work[goff+2+2N+k] = the group
+// of rank k, longest first; work[goff+2+3N] = the next item to hand out.
 __device__ __forceinline__ int *groups_n(const flide_tree_index &x, int goff) { return x.work + goff; }
 __device__ __forceinline__ int *groups_start(const flide_tree_index &x, int goff) {
   return x.work + goff + 1;
@@ -89,6 +91,13 @@ __device__ __forceinline__ int *groups_start(const flide_tree_index &x, int goff
 __device__ __forceinline__ int *groups_count(const flide_tree_index &x, int goff) {
   return x.work + goff + 2 + x.N;
 }
+__device__ __forceinline__ int *groups_order(const flide_tree_index &x, int goff) {
+  return x.work + goff + 2 + 2 * x.N;
+}
+__device__ __forceinline__ int *groups_next(const flide_tree_index &x, int goff) {
+  return x.work + goff + 2 + 3 * x.N;
+}
+constexpr int kMaxSortedGroups = 2048;  // more groups than this keep level order
 
 // Groups the nodes of one level: a root, a node with a state slot or a node
 // longer than a chunk is alone; consecutive leaves (consecutive ids) with the
@@ -98,7 +107,10 @@ __global__ void gdn_groups_kernel(flide_tree_index x, int level, int goff) {
   int *flag = groups_count(x, goff);  // temporary flags, then counts
   int *gstart = groups_start(x, goff);
   if (failed(x.status)) {
-    if (threadIdx.x == 0) *groups_n(x, goff) = 0;
+    if (threadIdx.x == 0) {
+      *groups_n(x, goff) = 0;
+      *groups_next(x, goff) = 0;
+    }
     return;
   }
   const int L0 = x.level_ptr[level], n = x.level_ptr[level + 1] - L0;
@@ -144,7 +156,30 @@ __global__ void gdn_groups_kernel(flide_tree_index x, int level, int goff) {
   // 4: counts
   for (int g = threadIdx.x; g < carry; g += blockDim.x)
     flag[g] = (g + 1 < carry ? gstart[g + 1] : n) - gstart[g];
-  if (threadIdx.x == 0) *groups_n(x, goff) = carry;
+  __syncthreads();
+  // 5: hand-out order, longest group (in tokens) first, so the persistent
+  //    CTAs' greedy pick-up of items stays balanced; ties keep level order
+  __shared__ int len[kMaxSortedGroups];
+  int *order = groups_order(x, goff);
+  if (carry <= kMaxSortedGroups) {
+    for (int g = threadIdx.x; g < carry; g += blockDim.x) {
+      const int first = x.level_node[L0 + gstart[g]], last = x.level_node[L0 + gstart[g] + flag[g] - 1];
+      len[g] = x.node_start[last + 1] - x.node_start[first];
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < carry; g += blockDim.x) {
+      const int lg = len[g];
+      int rank = 0;
+      for (int o = 0; o < carry; ++o) rank += (len[o] > lg) || (len[o] == lg && o < g);
+      order[rank] = g;
+    }
+  } else {
+    for (int g = threadIdx.x; g < carry; g += blockDim.x) order[g] = g;
+  }
+  if (threadIdx.x == 0) {
+    *groups_n(x, goff) = carry;
+    *groups_next(x, goff) = 0;
+  }
 }
 
 // Self-check: records the first failed bounds check (site, value) in the
@@ -228,8 +263,20 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     return __syncthreads_and(r);
   };
 
-  for (long it = blockIdx.x; ok && it < items; it += gridDim.x) {
-    const int grp = (int)(it / p.H), h = (int)(it % p.H);
+  int *s_item = reinterpret_cast<int *>(smem + SM_MISC + 8);
+  for (;;) {
+    // next (group, head) item from the level's shared counter
+    if (tid == 0) *s_item = atomicAdd(groups_next(x, p.goff), 1);
+    __syncthreads();
+    const long it = *s_item;
+    __syncthreads();
+    if (!ok || it >= items) break;
+    const int rk = (int)(it / p.H), h = (int)(it % p.H);
+    const int grp = groups_order(x, p.goff)[rk];
+    if (grp < 0 || grp >= n_groups) {
+      if (tid == 0) check_fail(x, 6, grp);
+      break;
+    }
     const int k0 = groups_start(x, p.goff)[grp], cnt = groups_count(x, p.goff)[grp];
     const int Nact = x.counts[FLIDE_CNT_N], Tact = x.counts[FLIDE_CNT_T];
     if (k0 < 0 || cnt < 1 || L0 + k0 + cnt > Nact) {

@@ -86,6 +86,29 @@ def fanout_tree(R: int, prefix: int, branches: int, branch_len: int,
     return _tree([(past, nodes)] * R, 1 if branches else 0)
 
 
+def warm_variant(tree: Tree):
+    """The same batch resumed from checkpoints: each root's tokens move into
+    its request's checkpointed past (past_len + root length) and the root keeps
+    zero tokens, so only branch tokens remain in the stream.  Returns the new
+    tree and the stream rows of the original tree that it keeps, in order.
+    With the original step's checkpoint (past rows then root rows per request,
+    and the root's end states) as past K/V and GDN state_in, the outputs of the
+    kept rows are the original ones (resume equals scratch)."""
+    rp, pa, sl, pl = tree.arrays()
+    starts = np.concatenate([[0], np.cumsum(sl)]).astype(np.int64)
+    reqs, keep = [], []
+    for r in range(tree.R):
+        n0, n1 = int(rp[r]), int(rp[r + 1])
+        if n1 == n0:
+            reqs.append((int(pl[r]), []))
+            continue
+        nodes = [(-1, 0)] + [(int(pa[n]), int(sl[n])) for n in range(n0 + 1, n1)]
+        reqs.append((int(pl[r]) + int(sl[n0]), nodes))
+        keep.append(np.arange(starts[n0 + 1], starts[n1]))
+    rows = np.concatenate(keep) if keep else np.zeros(0, np.int64)
+    return _tree(reqs, tree.levels), rows
+
+
 def leveled_tree(rng: np.random.Generator, R: int, depth_range=(1, 3),
                  options_range=(2, 256), prefix_range=(256, 8192),
                  branch_range=(4, 64), n_resume: int = 0,
