@@ -46,7 +46,7 @@ using namespace sm100;
 
 constexpr int C = 64;    // tokens per chunk
 constexpr int D = 128;   // dk = dv
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // two warps per TMEM lane group: warp w and w + 4 split the columns
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // shared-memory map, bytes from a 1024-aligned base
@@ -216,7 +216,9 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = smem_u32(smem);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int lg = warp & 3, wg = warp >> 2;  // TMEM lane group; column half
+  const int row = lg * 32 + lane;           // this thread's TMEM lane = tile row
   const flide_tree_index &x = p.x;
   float *sbeta = reinterpret_cast<float *>(smem + SM_SCAL);
   float *sG = sbeta + C;
@@ -242,7 +244,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+  const uint32_t tl = tmem + ((uint32_t)(lg * 32) << 16);  // this warp's TMEM lanes
   volatile int *vabort = abort_flag;
 
   const int n_groups = failed(x.status) ? 0 : *groups_n(x, p.goff);
@@ -316,18 +318,18 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       src = p.node_state + ((size_t)ps * p.H + h) * D * D;
     }
-    for (int half = 0; half < 2; ++half) {
+    {
       uint32_t v[64];
 #pragma unroll
       for (int i = 0; i < 64; i += 4) {
-        const float4 f4 = src ? *reinterpret_cast<const float4 *>(src + (size_t)tid * D + half * 64 + i)
+        const float4 f4 = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * D + wg * 64 + i)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
         v[i] = __float_as_uint(f4.x);
         v[i + 1] = __float_as_uint(f4.y);
         v[i + 2] = __float_as_uint(f4.z);
         v[i + 3] = __float_as_uint(f4.w);
       }
-      tmem_st64(tl + R_S + half * 64, v);
+      tmem_st64(tl + R_S + wg * 64, v);
     }
     tc_fence_before();
     __syncthreads();
@@ -432,25 +434,20 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __syncwarp();
       // ---- meanwhile: bf16 copy of S0 (B operand, rows = dv); rescale S
       {
-        uint32_t sr[128];
-        tmem_ld128(tl + R_S, sr);
-        uint8_t *s0 = smem + SM_S0;
+        uint32_t sr[64];
+        tmem_ld64(tl + R_S + wg * 64, sr);
+        uint8_t *s0 = smem + SM_S0 + wg * 16384;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < 8; ++q) {
           float f[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
-          st_chunk(s0 + (q >> 3) * 16384, tid, q & 7, pack8(f));
+          st_chunk(s0, row, q, pack8(f));
         }
         if (update) {
-          uint32_t a[64], b2[64];
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            a[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
-            b2[i] = __float_as_uint(__uint_as_float(sr[64 + i]) * gam_last);
-          }
-          tmem_st64(tl + R_S, a);
-          tmem_st64(tl + R_S + 64, b2);
+          for (int i = 0; i < 64; ++i) sr[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
+          tmem_st64(tl + R_S + wg * 64, sr);
         }
       }
       if (!mma_sync()) { ok = false; break; }
@@ -459,37 +456,36 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       //      entry (i, j) scaled by gamma_i / gamma_j = 2^(G2_i - G2_j) where
       //      j precedes (A) or equals (QK^T) i inside i's segment
       {
-        uint32_t d1[64];
-        tmem_ld32(tl + R1, *reinterpret_cast<uint32_t(*)[32]>(d1));
-        tmem_ld32(tl + R1 + 32, *reinterpret_cast<uint32_t(*)[32]>(d1 + 32));
-        const int i = tid & (C - 1);
-        const bool is_a = tid < C;
+        uint32_t d1[32];  // this warp's half of the row: j = 32 wg + u
+        tmem_ld32(tl + R1 + 32 * wg, d1);
+        const int i = row & (C - 1);
+        const bool is_a = row < C;
         const float G2i = sG2[i], scale_i = is_a ? sbeta[i] : 1.f;
         const int si = sseg[i];
         const int jmax = is_a ? i - 1 : i;  // last visible j
         const float4 *g4 = reinterpret_cast<const float4 *>(sG2);
         const int4 *s4 = reinterpret_cast<const int4 *>(sseg);
-        float e[64];
+        float e[32];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float4 gv = g4[q];
-          const int4 sv = s4[q];
+        for (int q = 0; q < 8; ++q) {
+          const float4 gv = g4[8 * wg + q];
+          const int4 sv = s4[8 * wg + q];
           const float gj[4] = {gv.x, gv.y, gv.z, gv.w};
           const int sj[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int j = 4 * q + u;
+            const int jj = 4 * q + u, j = 32 * wg + jj;
             const bool m = j <= jmax && sj[u] == si && si >= 0;
-            e[j] = m ? scale_i * ex2_approx(G2i - gj[u]) * __uint_as_float(d1[j]) : 0.f;
+            e[jj] = m ? scale_i * ex2_approx(G2i - gj[u]) * __uint_as_float(d1[jj]) : 0.f;
           }
         }
         if (is_a) {
 #pragma unroll
-          for (int j = 0; j < C; ++j) Am[i * A_LD + j] = e[j];
+          for (int jj = 0; jj < 32; ++jj) Am[i * A_LD + 32 * wg + jj] = e[jj];
         } else {
           uint8_t *pm = smem + SM_PM;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) st_chunk(pm, tid, q, pack8(e + 8 * q));  // token row i at tile row 64 + i
+          for (int q = 0; q < 4; ++q) st_chunk(pm, row, 4 * wg + q, pack8(e + 8 * q));  // token row i at tile row 64 + i
         }
       }
       __syncthreads();
@@ -519,81 +515,61 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         __syncthreads();
         // block row bi: X_bj = sum_{k=j}^{bi-1} A_bk T_kj, then T_bj = -T_bb X_bj.
-        // Thread -> (row r of the block row, column pair 2cp, 2cp+1) for every
-        // column block j < bi: up to six independent sums, each A value
-        // loaded once for two columns.
+        // Thread -> (row r of the block row, column cc) for every column block
+        // j < bi: up to three independent sums.
         {
-          const int r = tid >> 3, cp = tid & 7;
+          const int r = tid >> 4, cc = tid & 15;
           for (int bi = 1; bi < 4; ++bi) {
             const float *arow = Am + (16 * bi + r) * A_LD;
-            float acc[3][2];
-#pragma unroll
-            for (int jb = 0; jb < 3; ++jb) acc[jb][0] = acc[jb][1] = 0.f;
+            float acc[3] = {0.f, 0.f, 0.f};
 #pragma unroll
             for (int kb = 0; kb < 3; ++kb) {
               if (kb >= bi) break;
 #pragma unroll
               for (int m = 0; m < 16; ++m) {
                 const float a = arow[16 * kb + m];
-                const float *trow = Tm + (16 * kb + m) * A_LD + 2 * cp;
+                const float *trow = Tm + (16 * kb + m) * A_LD + cc;
 #pragma unroll
-                for (int jb = 0; jb < 3; ++jb) {
-                  if (jb <= kb) {
-                    acc[jb][0] = fmaf(a, trow[16 * jb], acc[jb][0]);
-                    acc[jb][1] = fmaf(a, trow[16 * jb + 1], acc[jb][1]);
-                  }
-                }
+                for (int jb = 0; jb < 3; ++jb)
+                  if (jb <= kb) acc[jb] = fmaf(a, trow[16 * jb], acc[jb]);
               }
             }
 #pragma unroll
-            for (int jb = 0; jb < 3; ++jb) {
-              if (jb < bi) {
-                Xm[(jb * 16 + r) * X_LD + 2 * cp] = acc[jb][0];
-                Xm[(jb * 16 + r) * X_LD + 2 * cp + 1] = acc[jb][1];
-              }
-            }
+            for (int jb = 0; jb < 3; ++jb)
+              if (jb < bi) Xm[(jb * 16 + r) * X_LD + cc] = acc[jb];
             __syncthreads();
             const float *trow = Tm + (16 * bi + r) * A_LD + 16 * bi;
-#pragma unroll
-            for (int jb = 0; jb < 3; ++jb) acc[jb][0] = acc[jb][1] = 0.f;
+            acc[0] = acc[1] = acc[2] = 0.f;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
               const float tv = m <= r ? trow[m] : 0.f;
 #pragma unroll
-              for (int jb = 0; jb < 3; ++jb) {
-                if (jb < bi) {
-                  acc[jb][0] = fmaf(tv, Xm[(jb * 16 + m) * X_LD + 2 * cp], acc[jb][0]);
-                  acc[jb][1] = fmaf(tv, Xm[(jb * 16 + m) * X_LD + 2 * cp + 1], acc[jb][1]);
-                }
-              }
+              for (int jb = 0; jb < 3; ++jb)
+                if (jb < bi) acc[jb] = fmaf(tv, Xm[(jb * 16 + m) * X_LD + cc], acc[jb]);
             }
 #pragma unroll
-            for (int jb = 0; jb < 3; ++jb) {
-              if (jb < bi) {
-                Tm[(16 * bi + r) * A_LD + 16 * jb + 2 * cp] = -acc[jb][0];
-                Tm[(16 * bi + r) * A_LD + 16 * jb + 2 * cp + 1] = -acc[jb][1];
-              }
-            }
+            for (int jb = 0; jb < 3; ++jb)
+              if (jb < bi) Tm[(16 * bi + r) * A_LD + 16 * jb + cc] = -acc[jb];
             __syncthreads();
           }
         }
         // T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles:
         // thread -> (row i, half of the columns)
         {
-          const int i = tid >> 1, hh = tid & 1;
+          const int i = tid >> 2, qq = tid & 3;  // row, quarter of the columns
           uint8_t *t1 = smem + SM_TA, *t2 = smem + SM_TA + 16384;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             float f1[8], f2[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              const int j = 32 * hh + 8 * q + u;
+              const int j = 16 * qq + 8 * q + u;
               const float tv = (j >> 4) <= (i >> 4) ? Tm[i * A_LD + j] : 0.f;
               f1[u] = tv * sbeta[j] * sgam[j];
               f2[u] = tv * sbeta[j];
             }
-            st_chunk(t1, i, 4 * hh + q, pack8(f1));
-            st_chunk(t2, i, 4 * hh + q, pack8(f2));
+            st_chunk(t1, i, 2 * qq + q, pack8(f1));
+            st_chunk(t2, i, 2 * qq + q, pack8(f2));
           }
         }
       }
@@ -615,16 +591,16 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!mma_sync()) { ok = false; break; }
 
       // ---- -W (token rows) as a K-major A operand over T' / T''
-      if (tid < C) {
-        uint32_t w[128];
-        tmem_ld128(tl + R2, w);
-        uint8_t *nw = smem + SM_TA;
+      if (row < C) {
+        uint32_t w[64];
+        tmem_ld64(tl + R2 + wg * 64, w);
+        uint8_t *nw = smem + SM_TA + wg * 16384;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < 8; ++q) {
           float f[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(w[8 * q + u]);
-          st_chunk(nw + (q >> 3) * 16384, tid, q & 7, pack8(f));
+          st_chunk(nw, row, q, pack8(f));
         }
       }
       fence_proxy_async_smem();
@@ -646,24 +622,24 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
       // ---- Delta rows (token j) -> MN-major B over S0's first half, and
       //      Delta'^T = (Delta * gamma_last/gamma_j)^T -> K-major A (second half)
-      if (tid < C) {
-        const int j = tid;
-        uint32_t dr[128];
-        tmem_ld128(tl + R3, dr);
-        uint8_t *db = smem + SM_S0;
+      if (row < C) {
+        const int j = row;  // token; this warp handles dv = 64 wg .. 64 wg + 63
+        uint32_t dr[64];
+        tmem_ld64(tl + R3 + wg * 64, dr);
+        uint8_t *db = smem + SM_S0 + wg * 8192;
         __nv_bfloat16 *dat = reinterpret_cast<__nv_bfloat16 *>(smem + SM_S0 + 16384);
         const float sc = gam_last / sgam[j];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < 8; ++q) {
           float f[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(dr[8 * q + u]);
-          st_chunk(db + (q >> 3) * 8192, j, q & 7, pack8(f));
+          st_chunk(db, j, q, pack8(f));
         }
         if (update) {
 #pragma unroll
-          for (int cdv = 0; cdv < D; ++cdv)
-            dat[sw_elem(cdv, j) >> 1] = __float2bfloat16_rn(__uint_as_float(dr[cdv]) * sc);
+          for (int c = 0; c < 64; ++c)
+            dat[sw_elem(64 * wg + c, j) >> 1] = __float2bfloat16_rn(__uint_as_float(dr[c]) * sc);
         }
       }
       fence_proxy_async_smem();
@@ -685,13 +661,13 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!mma_sync()) { ok = false; break; }
 
       // ---- outputs (token rows 64-127): o_i = gamma_i (Q S0^T)_i + ((M o QK^T) Delta)_i
-      if (tid >= C) {
-        const int i = tid - C;
+      if (row >= C) {
+        const int i = row - C;
         const bool valid = i < n && cbeg + i < Tact;
         __nv_bfloat16 *o = p.out + ((size_t)(cbeg + i) * p.H + h) * D;
         const float gi = sgam[i];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        {
+          const int half = wg;  // this warp's 64 output dims
           uint32_t o1[32], o2[32];
 #pragma unroll
           for (int qq = 0; qq < 2; ++qq) {
@@ -717,11 +693,11 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     // ---- end state of a node with a slot
     if (scan && slot >= 0) {
-      uint32_t sr[128];
-      tmem_ld128(tl + R_S, sr);
-      float *dst = p.node_state + ((size_t)slot * p.H + h) * D * D + (size_t)tid * D;
+      uint32_t sr[64];
+      tmem_ld64(tl + R_S + wg * 64, sr);
+      float *dst = p.node_state + ((size_t)slot * p.H + h) * D * D + (size_t)row * D + wg * 64;
 #pragma unroll
-      for (int i = 0; i < 128; i += 4)
+      for (int i = 0; i < 64; i += 4)
         *reinterpret_cast<float4 *>(dst + i) =
             make_float4(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1]),
                         __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
