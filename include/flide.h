@@ -266,6 +266,19 @@ int flide_state_resume(int32_t R, const int32_t *src_req, int32_t src_R,
                        void *past_v, int32_t past_rows, float *state_in,
                        int32_t *status, flide_stream stream);
 
+/* Diagnostic, with no counterpart in the pages: runs, in one thread on
+ * `stream`, the bounded mbarrier wait that every kernel of this library uses
+ * (try_wait with a suspend hint, limit checked against the global timer) on a
+ * barrier in shared memory that nothing arrives at, with a limit of
+ * timeout_us microseconds (1 .. 10,000,000).  On expiry it writes
+ * FLIDE_ERR_TIMEOUT to *status (device int32) and returns, leaving the
+ * context usable.  With arrive != 0 the thread first arrives on the barrier
+ * itself, so the wait completes at once and *status is left unchanged (the
+ * control case).  Returns FLIDE_ERR_SHAPE for a null status or a limit out of
+ * range. */
+int flide_selftest_wait_timeout(int32_t *status, int32_t timeout_us, int32_t arrive,
+                                flide_stream stream);
+
 /* Static message for a status code. */
 const char *flide_strerror(int32_t code);
 

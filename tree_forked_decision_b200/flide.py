@@ -29,7 +29,7 @@ INDEX_ARRAYS = ["status", "counts", "node_start", "node_req", "depth", "anc_ptr"
 # every extern "C" symbol declared in include/flide.h
 SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build",
            "flide_fork_attn", "flide_fork_attn_noalloc", "flide_fork_gdn", "flide_state_save",
-           "flide_state_resume", "flide_strerror"]
+           "flide_state_resume", "flide_selftest_wait_timeout", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -83,6 +83,8 @@ def _lib():
         lib.flide_state_resume.argtypes = [I32, P, I32, P, P, P, P, I32, I32, I32, I32, I32, I32,
                                            P, P, P, I32, P, P, P]
         lib.flide_state_resume.restype = ctypes.c_int
+        lib.flide_selftest_wait_timeout.argtypes = [P, I32, I32, P]
+        lib.flide_selftest_wait_timeout.restype = ctypes.c_int
         lib.flide_strerror.argtypes = [ctypes.c_int32]
         lib.flide_strerror.restype = ctypes.c_char_p
         _LIB = lib
@@ -258,3 +260,12 @@ def state_resume(src_req, src_ckpt_start, src_k, src_v, src_S, past_len, past_k,
                                      past_k.shape[0], _ptr(state_in), _ptr(status),
                                      _stream(stream)),
            "flide_state_resume")
+
+
+def selftest_wait_timeout(status, timeout_us: int, arrive: bool = False, stream=None):
+    """The library's bounded device wait on a barrier nothing arrives at
+    (diagnostic): FLIDE_ERR_TIMEOUT lands in `status` after `timeout_us`; with
+    arrive=True the wait completes at once and `status` is left alone."""
+    _check(_lib().flide_selftest_wait_timeout(_ptr(status), int(timeout_us), 1 if arrive else 0,
+                                              _stream(stream)),
+           "flide_selftest_wait_timeout")
