@@ -609,6 +609,19 @@ def main():
                 "avg_launch_ms": attn_ms,
             }
 
+    # combined roofline of the step: the layers' roofline times summed, over the
+    # measured per-step P50
+    combined = None
+    parts = {}
+    if a is not None:
+        parts["fork_attn_ms"] = 1000.0 * attn_work(tree, a)[0] / (peak * 1e12)
+    if g is not None:
+        parts["fork_gdn_ms"] = 1000.0 * gdn_work(tree, g, step.slots) / (hbm * 1e9)
+    if parts:
+        rt = sum(parts.values())
+        combined = {"roofline_ms": rt, "measured_p50_ms": p50_ms, "frac": rt / p50_ms, "parts": parts,
+                    "peaks": "attention: sustained dense bf16; GDN: HBM copy (measured)"}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, desc, threads = cpu_oracle_rate(tree, a, g, args.cpu_rows, args.cpu_pairs)
@@ -626,6 +639,7 @@ def main():
                    "l2": "inputs larger than L2 (GBs per step), no flush",
                    "parallelism": f"dp{ws} (independent requests per rank)", "seed": seed},
         "roofline": roofline,
+        "roofline_combined": combined,
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
