@@ -189,3 +189,6 @@ def gdn(tree, q, k, v, g, beta, state_in=None, memoise=True, pairs=None,
     if st != OK:
         raise OracleError(st)
     return (out, states) if want_states else out
+
+
+from .decision import branch_logprob, option_probs, tvd  # noqa: E402,F401  (numpy, fp64)
