@@ -266,6 +266,39 @@ int flide_state_resume(int32_t R, const int32_t *src_req, int32_t src_R,
                        void *past_v, int32_t past_rows, float *state_in,
                        int32_t *status, flide_stream stream);
 
+/* ---- decision scoring (next step after the layers) -------------------------
+ * Decision models answer with probabilities over a few candidate options
+ * (openai-hub.com news article on the Flide release, paragraphs on Jev-like
+ * decision models); engines are compared by total variation distance to a
+ * high-precision reference (kongchang.com article on Flide, "total variation
+ * distance" box).  Reading used: each leaf of a request's tree is an option
+ * scored by the log-likelihood of its path's branch tokens under an LM head,
+ * and the decision is the softmax over the request's leaves.
+ *
+ * Bytes of `workspace` that flide_branch_logprob needs for a tree of up to T
+ * stream tokens and a vocabulary of V (partial sums of the vocabulary split). */
+size_t flide_branch_logprob_workspace_bytes(int32_t T, int32_t V);
+
+/* log p_t = h_t . w_{y_t} - logsumexp_v h_t . w_v for every branch token t
+ * (tokens of non-root nodes); root tokens get NaN.
+ *   h [T, D] bf16 hidden states (row t = stream token t), w_lm [V, D] bf16,
+ *   targets [T] int32 in [0, V) (read for branch tokens only), logp [T] fp32 out,
+ *   workspace of flide_branch_logprob_workspace_bytes(idx->T, V) bytes (device).
+ * D % 64 == 0, V % 128 == 0, dtype FLIDE_BF16 (fp32 accumulation) else
+ * FLIDE_ERR_SHAPE; idx built by flide_tree_build; uses idx->work.  Device errors
+ * (expired waits) land in idx->status. */
+int flide_branch_logprob(const void *h, const void *w_lm, const int32_t *targets,
+                         const flide_tree_index *idx, int32_t D, int32_t V, int32_t dtype,
+                         float *logp, void *workspace, size_t workspace_bytes,
+                         flide_stream stream);
+
+/* Per node: path_logp[n] = sum of logp over the branch tokens from the root's
+ * child down to n (0 for roots); prob[n] = softmax of path_logp over the leaves
+ * of n's request for leaves, 0 for other nodes.  logp [T] fp32 (from
+ * flide_branch_logprob), path_logp and prob [N] fp32 out (device). */
+int flide_option_probs(const flide_tree_index *idx, const float *logp, float *path_logp,
+                       float *prob, flide_stream stream);
+
 /* Diagnostic, with no counterpart in the pages: runs, in one thread on
  * `stream`, the bounded mbarrier wait that every kernel of this library uses
  * (try_wait with a suspend hint, limit checked against the global timer) on a

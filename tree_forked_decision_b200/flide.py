@@ -29,7 +29,8 @@ INDEX_ARRAYS = ["status", "counts", "node_start", "node_req", "depth", "anc_ptr"
 # every extern "C" symbol declared in include/flide.h
 SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build",
            "flide_fork_attn", "flide_fork_attn_noalloc", "flide_fork_gdn", "flide_state_save",
-           "flide_state_resume", "flide_selftest_wait_timeout", "flide_strerror"]
+           "flide_state_resume", "flide_branch_logprob_workspace_bytes", "flide_branch_logprob",
+           "flide_option_probs", "flide_selftest_wait_timeout", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -83,6 +84,12 @@ def _lib():
         lib.flide_state_resume.argtypes = [I32, P, I32, P, P, P, P, I32, I32, I32, I32, I32, I32,
                                            P, P, P, I32, P, P, P]
         lib.flide_state_resume.restype = ctypes.c_int
+        lib.flide_branch_logprob_workspace_bytes.argtypes = [I32, I32]
+        lib.flide_branch_logprob_workspace_bytes.restype = ctypes.c_size_t
+        lib.flide_branch_logprob.argtypes = [P, P, P, P, I32, I32, I32, P, P, ctypes.c_size_t, P]
+        lib.flide_branch_logprob.restype = ctypes.c_int
+        lib.flide_option_probs.argtypes = [P, P, P, P, P]
+        lib.flide_option_probs.restype = ctypes.c_int
         lib.flide_selftest_wait_timeout.argtypes = [P, I32, I32, P]
         lib.flide_selftest_wait_timeout.restype = ctypes.c_int
         lib.flide_strerror.argtypes = [ctypes.c_int32]
@@ -269,3 +276,39 @@ def selftest_wait_timeout(status, timeout_us: int, arrive: bool = False, stream=
     _check(_lib().flide_selftest_wait_timeout(_ptr(status), int(timeout_us), 1 if arrive else 0,
                                               _stream(stream)),
            "flide_selftest_wait_timeout")
+
+
+def branch_logprob_workspace(index: TreeIndex, V: int, device="cuda") -> torch.Tensor:
+    n = int(_lib().flide_branch_logprob_workspace_bytes(index.T, int(V)))
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+
+
+def branch_logprob(h, w_lm, targets, index: TreeIndex, logp=None, workspace=None, stream=None):
+    """log p(target) of every branch token under the LM head w_lm [V, D];
+    h [T, D] (or [T, heads, dim]) bf16, targets [T] int32.  Root tokens: NaN."""
+    T = h.shape[0]
+    D = h[0].numel()
+    V = w_lm.shape[0]
+    if logp is None:
+        logp = torch.empty(T, dtype=torch.float32, device=h.device)
+    if workspace is None:
+        workspace = branch_logprob_workspace(index, V, device=h.device)
+    _check(_lib().flide_branch_logprob(_ptr(h), _ptr(w_lm), _ptr(targets), ctypes.byref(index.c), D, V,
+                                       _dtype_code(h), _ptr(logp), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
+           "flide_branch_logprob")
+    return logp
+
+
+def option_probs(index: TreeIndex, logp, path_logp=None, prob=None, stream=None):
+    """Per node: path log-likelihood and, for leaves, the softmax over the
+    request's leaves (the decision distribution)."""
+    N = index.N
+    if path_logp is None:
+        path_logp = torch.empty(max(N, 1), dtype=torch.float32, device=logp.device)
+    if prob is None:
+        prob = torch.empty(max(N, 1), dtype=torch.float32, device=logp.device)
+    _check(_lib().flide_option_probs(ctypes.byref(index.c), _ptr(logp), _ptr(path_logp), _ptr(prob),
+                                     _stream(stream)),
+           "flide_option_probs")
+    return path_logp, prob
