@@ -375,6 +375,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--no-warm", action="store_true", help="skip the resumed-prefix (warm) timing")
+    ap.add_argument("--no-decision", action="store_true", help="skip the decision-scoring timing")
+    ap.add_argument("--vocab", type=int, default=8192, help="LM-head vocabulary of the decision leg")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--cpu-pairs", type=int, default=16)
     ap.add_argument("--ref-rows", type=int, default=2000)
@@ -609,6 +611,44 @@ def main():
                 "avg_launch_ms": attn_ms,
             }
 
+    # decision scoring on the step's attention output: log p of every branch
+    # token under a random LM head, then the softmax over each request's options
+    decision = None
+    if not args.no_decision and a is not None and a["q"].dtype == torch.bfloat16 and tree.branch_tokens:
+        D, V = step.o[0].numel(), args.vocab
+        grng = torch.Generator(device="cpu").manual_seed(seed + 17)
+        w_lm = (torch.randn((V, D), generator=grng) / math.sqrt(D)).to(torch.bfloat16).to(device)
+        y = torch.randint(0, V, (tree.T,), generator=grng, dtype=torch.int32).to(device)
+        h = step.o.view(tree.T, D)
+        lp = torch.empty(tree.T, dtype=torch.float32, device=device)
+        ws_buf = flide.branch_logprob_workspace(step.idx, V, device=device)
+        pth = torch.empty(max(tree.N, 1), dtype=torch.float32, device=device)
+        prb = torch.empty_like(pth)
+
+        def dec_step():
+            flide.branch_logprob(h, w_lm, y, step.idx, logp=lp, workspace=ws_buf)
+            flide.option_probs(step.idx, lp, path_logp=pth, prob=prb)
+
+        for _ in range(max(args.warmup, 1)):
+            dec_step()
+        dev_ = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            dev_[i][0].record()
+            dec_step()
+            dev_[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        if step.idx.status() != 0:
+            raise SystemExit(f"device status {step.idx.status()} in the decision leg")
+        d_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in dev_), pg, device)
+        dflops = 2.0 * tree.branch_tokens * D * V
+        decision = {"ms": d_ms, "tflops": dflops / (d_ms / 1000.0) / 1e12,
+                    "frac_of_tensor_peak": dflops / (d_ms / 1000.0) / 1e12 / peak,
+                    "algorithmic_flops": dflops, "D": D, "V": V, "options": int(np.sum(prb[:tree.N].cpu().numpy() > 0)),
+                    "note": "log p of every branch token under a random bf16 LM head on the attention "
+                            "output, path sums and softmax over each request's leaves"}
+
     # combined roofline of the step: the layers' roofline times summed, over the
     # measured per-step P50
     combined = None
@@ -646,6 +686,7 @@ def main():
         "p50_ms": p50_ms, "p95_ms": p95_ms,
         "graph": graph,
         "warm": warm,
+        "decision": decision,
         "gpu_launches": step.launches * args.steps,
         "clocks": clk.summary(),
     }
