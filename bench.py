@@ -68,22 +68,24 @@ def attn_work(tree, a):
     return flops, byts
 
 
-def gdn_work(tree, g, slots):
+def gdn_work(tree, g):
     """Algorithmic bytes of one GDN fork scan: q, k, v, out, g, beta once, one
-    fp32 state write per saved node, and one state read per parent with
-    children (its checkpoint is broadcast to all its branches) and per resumed
-    root."""
+    fp32 state write per saved node (roots and nodes with children), and one
+    state read per parent with children (its checkpoint is broadcast to all
+    its branches) and per resumed root."""
     H, dk, dv = g["H"], g["dk"], g["dv"]
     es = 2 if g["q"].dtype == torch.bfloat16 else 4
     state = 4 * H * dk * dv
     has_child = np.zeros(tree.N, bool)
+    rp = tree.req_node_ptr
     for r in range(tree.R):
-        for n in range(tree.req_node_ptr[r], tree.req_node_ptr[r + 1]):
+        for n in range(rp[r], rp[r + 1]):
             if tree.parent[n] >= 0:
-                has_child[tree.req_node_ptr[r] + tree.parent[n]] = True
+                has_child[rp[r] + tree.parent[n]] = True
+    roots = int(np.sum(rp[1:] > rp[:-1]))
+    writes = int(has_child.sum()) + roots - int(sum(has_child[rp[r]] for r in range(tree.R) if rp[r + 1] > rp[r]))
     reads = int(has_child.sum()) + int(np.sum(tree.past_len > 0))
-    byts = tree.T * H * ((2 * dk + 2 * dv) * es + 8) + state * (slots + reads)
-    return byts
+    return tree.T * H * ((2 * dk + 2 * dv) * es + 8) + state * (writes + reads)
 
 
 # ---------------------------------------------------------------------------
@@ -122,15 +124,9 @@ class Step:
         self.gg, self.gb = dev(g["g"]), dev(g["beta"])
         self.state_in = dev(g["state_in"]) if np.any(tree.past_len > 0) else None
         self.go = torch.empty((tree.T, g["H"], g["dv"]), dtype=self.gq.dtype, device=device)
-        # node-state capacity: roots + every node that has children
-        has_child = np.zeros(tree.N, bool)
-        rp = tree.req_node_ptr
-        for r in range(tree.R):
-            for n in range(rp[r] + 1, rp[r + 1]):
-                has_child[rp[r] + tree.parent[n]] = True
-        roots = rp[:-1][rp[:-1] < rp[1:]]
-        has_child[roots] = True
-        self.slots = max(int(has_child.sum()), 1)
+        # node-state capacity: the slots the tree index assigns (roots, plus
+        # the inner nodes of the widest odd and even depth)
+        self.slots = max(flide.state_slots(tree), 1)
         self.node_state = torch.empty((self.slots, g["H"], g["dv"], g["dk"]), dtype=torch.float32,
                                       device=device)
         self.cS = torch.empty((tree.R, g["H"], g["dv"], g["dk"]), dtype=torch.float32, device=device)
@@ -585,7 +581,7 @@ def main():
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     kernels, roofline = {}, None
     if g is not None:
-        gbytes = gdn_work(tree, g, step.slots)
+        gbytes = gdn_work(tree, g)
         gdn_gbs = gbytes / (gdn_ms / 1000.0) / 1e9
         kernels["fork_gdn"] = {"ms": gdn_ms, "algorithmic_bytes": gbytes, "gbs": gdn_gbs,
                                "frac_of_hbm_peak": gdn_gbs / hbm, "bound": "hbm"}
@@ -656,7 +652,7 @@ def main():
     if a is not None:
         parts["fork_attn_ms"] = 1000.0 * attn_work(tree, a)[0] / (peak * 1e12)
     if g is not None:
-        parts["fork_gdn_ms"] = 1000.0 * gdn_work(tree, g, step.slots) / (hbm * 1e9)
+        parts["fork_gdn_ms"] = 1000.0 * gdn_work(tree, g) / (hbm * 1e9)
     if parts:
         rt = sum(parts.values())
         combined = {"roofline_ms": rt, "measured_p50_ms": p50_ms, "frac": rt / p50_ms, "parts": parts,

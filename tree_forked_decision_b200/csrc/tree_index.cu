@@ -143,24 +143,60 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
   }
   for (int lvl = D + 1 + tid; lvl <= x.max_depth + 1; lvl += blockDim.x) x.level_ptr[lvl] = N;
 
-  // state slots: roots and nodes that have children
+  // State slots.  A root keeps its slot for the whole call (its end state is
+  // the request's checkpoint).  An inner node at depth L >= 1 is read only by
+  // the depth-(L+1) launch, so inner nodes of odd depths share one region and
+  // those of even depths another, each sized by its largest level: depth L's
+  // slots are rewritten at depth L+2, after depth L+1 has read them.  Leaves
+  // have no slot.
   for (int n = tid; n < N; n += blockDim.x) x.state_slot[n] = 0;
   __syncthreads();
   for (int n = tid; n < N; n += blockDim.x) {
     int p = d.parent[n];
-    if (p >= 0) x.state_slot[rp[x.node_req[n]] + p] = 1;
+    if (p >= 0) x.state_slot[rp[x.node_req[n]] + p] = 1;  // has children
   }
   __syncthreads();
-  int slots = 0;
-  for (int b = 0; b < N; b += blockDim.x) {
-    int n = b + tid;
-    int f = 0;
-    if (n < N) f = (x.depth[n] == 0 || x.state_slot[n]) ? 1 : 0;
-    int tot;
-    int ex = block_excl_scan(f, scratch, &tot);
-    if (n < N) x.state_slot[n] = f ? slots + ex : -1;
-    slots += tot;
+  // inner nodes per level (L >= 1), for the two regions' sizes
+  int size_odd = 0, size_even = 0;
+  for (int lvl = 1; lvl <= D; ++lvl) {
+    const int a0 = x.level_ptr[lvl], a1 = x.level_ptr[lvl + 1];
+    int cnt = 0;
+    for (int b = a0; b < a1; b += blockDim.x) {
+      const int k = b + tid;
+      const int f = (k < a1 && x.state_slot[x.level_node[k]] == 1) ? 1 : 0;
+      int tot;
+      block_excl_scan(f, scratch, &tot);
+      cnt += tot;
+    }
+    if (lvl & 1) size_odd = max(size_odd, cnt); else size_even = max(size_even, cnt);
   }
+  // roots first, in level order (depth 0 is one level)
+  int roots = 0;
+  {
+    const int a0 = x.level_ptr[0], a1 = x.level_ptr[1];
+    for (int b = a0; b < a1; b += blockDim.x) {
+      const int k = b + tid;
+      int tot;
+      const int ex = block_excl_scan(k < a1 ? 1 : 0, scratch, &tot);
+      if (k < a1) x.state_slot[x.level_node[k]] = roots + ex;
+      roots += tot;
+    }
+  }
+  for (int lvl = 1; lvl <= D; ++lvl) {
+    const int a0 = x.level_ptr[lvl], a1 = x.level_ptr[lvl + 1];
+    const int base = roots + ((lvl & 1) ? 0 : size_odd);
+    int carry = 0;
+    for (int b = a0; b < a1; b += blockDim.x) {
+      const int k = b + tid;
+      const int n = k < a1 ? x.level_node[k] : -1;
+      const int f = (n >= 0 && x.state_slot[n] == 1) ? 1 : 0;
+      int tot;
+      const int ex = block_excl_scan(f, scratch, &tot);
+      if (n >= 0) x.state_slot[n] = f ? base + carry + ex : -1;
+      carry += tot;
+    }
+  }
+  const int slots = roots + size_odd + size_even;
 
   // checkpoint rows: past + root tokens of every request
   const int C = block_scan_array(R, [&](int r) {

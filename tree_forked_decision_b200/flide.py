@@ -312,3 +312,28 @@ def option_probs(index: TreeIndex, logp, path_logp=None, prob=None, stream=None)
                                      _stream(stream)),
            "flide_option_probs")
     return path_logp, prob
+
+
+def state_slots(tree) -> int:
+    """Node-state slots that flide_tree_build assigns to a tree (counts["SLOTS"]):
+    one per request root, plus the largest number of inner nodes (nodes with
+    children) at any odd depth and at any even depth >= 2 -- inner nodes of
+    depth L share their region with depth L+2, which is written only after
+    depth L+1 has read them."""
+    rp, parent, _seg, _past = tree.arrays()
+    R = len(rp) - 1
+    roots = int(sum(1 for r in range(R) if rp[r + 1] > rp[r]))
+    depth, inner = {}, set()
+    for r in range(R):
+        for n in range(rp[r], rp[r + 1]):
+            p = int(parent[n])
+            depth[n] = 0 if p < 0 else depth[rp[r] + p] + 1
+            if p >= 0:
+                inner.add(int(rp[r] + p))
+    per = {}
+    for n in inner:
+        if depth[n] >= 1:
+            per[depth[n]] = per.get(depth[n], 0) + 1
+    odd = max([c for d, c in per.items() if d % 2 == 1], default=0)
+    even = max([c for d, c in per.items() if d % 2 == 0], default=0)
+    return roots + odd + even
