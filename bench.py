@@ -372,6 +372,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--no-warm", action="store_true", help="skip the resumed-prefix (warm) timing")
     ap.add_argument("--no-decision", action="store_true", help="skip the decision-scoring timing")
+    ap.add_argument("--no-history", action="store_true", help="skip the paged history store timing")
     ap.add_argument("--vocab", type=int, default=8192, help="LM-head vocabulary of the decision leg")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--cpu-pairs", type=int, default=16)
@@ -645,6 +646,44 @@ def main():
                     "note": "log p of every branch token under a random bf16 LM head on the attention "
                             "output, path sums and softmax over each request's leaves"}
 
+    # the paged history store: append the step's roots (rows + end states) and
+    # gather the histories back as the next step's past (copies: HBM-bound)
+    history = None
+    if not args.no_history and a is not None and tree.root_tokens > 0:
+        from tree_forked_decision_b200.history import HistoryStore
+        brows = 256
+        nb = sum(-(-int(tree.seg_len[tree.req_node_ptr[r]]) // brows)
+                 for r in range(tree.R) if tree.req_node_ptr[r + 1] > tree.req_node_ptr[r]) + tree.R
+        gd = g if g is not None else {"H": 0, "dk": 0, "dv": 0}
+        store = HistoryStore(nb, brows, tree.R, nb, a["Hkv"], a["d"], H=gd["H"], dk=gd["dk"],
+                             dv=gd["dv"], dtype=step.k.dtype, device=device)
+        slots = list(range(tree.R))
+        ns = step.node_state if g is not None else None
+        store.commit(slots, tree, step.idx, step.k, step.v, ns)
+        store.resume(slots)
+        torch.cuda.synchronize()
+        hev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            hev[i][0].record()
+            store.resume(slots)
+            hev[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        if int(store.status.item()) != 0:
+            raise SystemExit(f"history store status {int(store.status.item())}")
+        h_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in hev), pg, device)
+        rows = sum(store.length(s_) for s_ in slots)
+        row_b = a["Hkv"] * a["d"] * step.k.element_size()
+        st_b = 4 * gd["H"] * gd["dk"] * gd["dv"] * tree.R
+        hbytes = 2 * (2 * rows * row_b) + 2 * st_b  # read + write of K, V rows and states
+        history = {"gather_ms": h_ms, "rows": rows, "block_rows": brows, "bytes": hbytes,
+                   "gbs": hbytes / (h_ms / 1000.0) / 1e9,
+                   "frac_of_hbm_peak": hbytes / (h_ms / 1000.0) / 1e9 / hbm,
+                   "note": "resume of every request's history (roots of this step) from the block pool "
+                           "into packed past K/V and GDN state_in"}
+        del store
+
     # combined roofline of the step: the layers' roofline times summed, over the
     # measured per-step P50
     combined = None
@@ -683,6 +722,7 @@ def main():
         "graph": graph,
         "warm": warm,
         "decision": decision,
+        "history": history,
         "gpu_launches": step.launches * args.steps,
         "clocks": clk.summary(),
     }

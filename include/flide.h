@@ -299,6 +299,64 @@ int flide_branch_logprob(const void *h, const void *w_lm, const int32_t *targets
 int flide_option_probs(const flide_tree_index *idx, const float *logp, float *path_logp,
                        float *prob, flide_stream stream);
 
+/* ---- multi-step agent history in a block-paged checkpoint pool -----------
+ * (kongchang.com article on Flide, closing section: growing agent histories
+ * and checkpoint reuse.)  Every request slot keeps its history's K/V rows in
+ * blocks of block_rows rows drawn from a shared free list, and its latest GDN
+ * state in state slot `slot` of a caller-owned state pool.  The host object
+ * below only does the bookkeeping; the pool memory itself is caller-owned
+ * device memory:
+ *   pool_k, pool_v [n_blocks * block_rows, Hkv, d]; pool_S [max_requests, H, dv, dk] fp32.
+ * The block table is [max_requests][max_blocks_per_request] int32 (-1 = none);
+ * copy it (flide_pool_export) to the device before append/gather. */
+typedef struct flide_pool flide_pool;
+
+/* Host allocator; NULL on bad arguments or out of host memory. */
+flide_pool *flide_pool_create(int32_t n_blocks, int32_t block_rows, int32_t max_requests,
+                              int32_t max_blocks_per_request);
+void flide_pool_destroy(flide_pool *pool);
+/* Reserves n more rows for request `slot` (blocks are taken from the free
+ * list as needed) and returns the history row where they start (its length
+ * before the call); -FLIDE_ERR_CAPACITY when blocks run out or the request's
+ * table is full, -FLIDE_ERR_INVALID for a bad slot.  Nothing changes on error. */
+int64_t flide_pool_append(flide_pool *pool, int32_t slot, int32_t n);
+/* Returns all blocks of request `slot` to the free list; its length becomes 0. */
+int flide_pool_release(flide_pool *pool, int32_t slot);
+/* History rows held by `slot` (negative status for a bad slot). */
+int32_t flide_pool_length(const flide_pool *pool, int32_t slot);
+int32_t flide_pool_free_blocks(const flide_pool *pool);
+/* Copies the block table [max_requests * max_blocks_per_request] and the
+ * lengths [max_requests] into host arrays. */
+int flide_pool_export(const flide_pool *pool, int32_t *table, int32_t *lengths);
+
+/* After a step: request r of the batch (req_slot[r] >= 0) writes its root's
+ * tokens (stream rows of its root node, k/v [T, Hkv, d]) to history rows
+ * [start[r], start[r] + root length) of its slot through the block table, and
+ * its root's end state node_state[state_slot[root]] to pool_S[req_slot[r]]
+ * (when node_state and pool_S are given).  start[r] is what flide_pool_append
+ * returned.  A row without a block sets FLIDE_ERR_CAPACITY in idx->status.
+ * All arrays are device memory; row bytes (Hkv d element size) % 16 == 0. */
+int flide_history_append(const flide_tree_index *idx, const int32_t *req_slot,
+                         const int32_t *start, const int32_t *table, int32_t max_blocks,
+                         int32_t block_rows, const void *k, const void *v, void *pool_k,
+                         void *pool_v, int32_t Hkv, int32_t d, int32_t dtype,
+                         const float *node_state, int32_t H, int32_t dk, int32_t dv,
+                         float *pool_S, flide_stream stream);
+
+/* Before a step: for the batch's R requests (req_slot[r] = pool slot, or -1 for
+ * a request with no history) writes past_len[r] = hist_len[slot], the
+ * histories' rows packed in request order into past_k/past_v [past_rows, Hkv, d]
+ * and state_in[r] = pool_S[slot] (zeros for -1) when state_in is given.
+ * Device errors to *status: FLIDE_ERR_CAPACITY when the rows exceed
+ * past_rows, FLIDE_ERR_INVALID for a slot >= max_requests or a row without a
+ * block.  R <= 4096. */
+int flide_history_gather(int32_t R, const int32_t *req_slot, int32_t max_requests,
+                         const int32_t *hist_len, const int32_t *table, int32_t max_blocks,
+                         int32_t block_rows, const void *pool_k, const void *pool_v, int32_t Hkv,
+                         int32_t d, int32_t dtype, const float *pool_S, int32_t H, int32_t dk,
+                         int32_t dv, int32_t *past_len, void *past_k, void *past_v,
+                         int32_t past_rows, float *state_in, int32_t *status, flide_stream stream);
+
 /* Diagnostic, with no counterpart in the pages: runs, in one thread on
  * `stream`, the bounded mbarrier wait that every kernel of this library uses
  * (try_wait with a suspend hint, limit checked against the global timer) on a

@@ -30,7 +30,10 @@ INDEX_ARRAYS = ["status", "counts", "node_start", "node_req", "depth", "anc_ptr"
 SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build",
            "flide_fork_attn", "flide_fork_attn_noalloc", "flide_fork_gdn", "flide_state_save",
            "flide_state_resume", "flide_branch_logprob_workspace_bytes", "flide_branch_logprob",
-           "flide_option_probs", "flide_selftest_wait_timeout", "flide_strerror"]
+           "flide_option_probs", "flide_pool_create", "flide_pool_destroy", "flide_pool_append",
+           "flide_pool_release", "flide_pool_length", "flide_pool_free_blocks", "flide_pool_export",
+           "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
+           "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -90,6 +93,26 @@ def _lib():
         lib.flide_branch_logprob.restype = ctypes.c_int
         lib.flide_option_probs.argtypes = [P, P, P, P, P]
         lib.flide_option_probs.restype = ctypes.c_int
+        lib.flide_pool_create.argtypes = [I32, I32, I32, I32]
+        lib.flide_pool_create.restype = P
+        lib.flide_pool_destroy.argtypes = [P]
+        lib.flide_pool_destroy.restype = None
+        lib.flide_pool_append.argtypes = [P, I32, I32]
+        lib.flide_pool_append.restype = ctypes.c_int64
+        lib.flide_pool_release.argtypes = [P, I32]
+        lib.flide_pool_release.restype = ctypes.c_int
+        lib.flide_pool_length.argtypes = [P, I32]
+        lib.flide_pool_length.restype = ctypes.c_int32
+        lib.flide_pool_free_blocks.argtypes = [P]
+        lib.flide_pool_free_blocks.restype = ctypes.c_int32
+        lib.flide_pool_export.argtypes = [P, P, P]
+        lib.flide_pool_export.restype = ctypes.c_int
+        lib.flide_history_append.argtypes = [P, P, P, P, I32, I32, P, P, P, P, I32, I32, I32, P,
+                                             I32, I32, I32, P, P]
+        lib.flide_history_append.restype = ctypes.c_int
+        lib.flide_history_gather.argtypes = [I32, P, I32, P, P, I32, I32, P, P, I32, I32, I32, P,
+                                             I32, I32, I32, P, P, P, I32, P, P, P]
+        lib.flide_history_gather.restype = ctypes.c_int
         lib.flide_selftest_wait_timeout.argtypes = [P, I32, I32, P]
         lib.flide_selftest_wait_timeout.restype = ctypes.c_int
         lib.flide_strerror.argtypes = [ctypes.c_int32]
