@@ -41,10 +41,22 @@ __device__ __forceinline__ int upper_bound_h(const int32_t *a, int n, int key) {
   return lo;
 }
 
-// one row of `bytes` (a multiple of 16) by the lanes of a warp
+// one row of `bytes` (a multiple of 16) by the lanes of a warp; up to four
+// 16-byte loads per lane are issued before their stores
 __device__ __forceinline__ void copy_row16(char *dst, const char *src, int bytes, int lane) {
-  for (int o = lane * 16; o < bytes; o += 32 * 16)
-    *reinterpret_cast<uint4 *>(dst + o) = *reinterpret_cast<const uint4 *>(src + o);
+  for (int o0 = lane * 16; o0 < bytes; o0 += 4 * 32 * 16) {
+    uint4 t[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int o = o0 + u * 32 * 16;
+      if (o < bytes) t[u] = __ldg(reinterpret_cast<const uint4 *>(src + o));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int o = o0 + u * 32 * 16;
+      if (o < bytes) *reinterpret_cast<uint4 *>(dst + o) = t[u];
+    }
+  }
 }
 
 // physical pool row of logical history row `row` of pool slot `s`, or -1
