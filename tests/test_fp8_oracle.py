@@ -1,0 +1,136 @@
+"""Pins of the e4m3 oracle (oracle/fp8.py) against things other than itself:
+the format's defining values (OCP 8-bit floating point specification, e4m3),
+PyTorch's own float8_e4m3fn conversion (a library routine) over every code and
+over random in-range values, round-half-to-even ties, saturation, the
+per-tensor scaling steps, and a brute-force fp64 attention on a tiny tree."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import fp8
+
+
+def test_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = fp8.decode_e4m3(codes)
+    assert np.array_equal(got, want, equal_nan=True)
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6),
+    (0x38, 1.0), (0x39, 1.125), (0x40, 2.0), (0x7E, 448.0), (0xB8, -1.0), (0xFE, -448.0),
+])
+def test_decode_defining_values(code, value):
+    assert fp8.decode_e4m3(np.array([code], np.uint8))[0] == value
+
+
+def test_nan_codes():
+    v = fp8.decode_e4m3(np.array([0x7F, 0xFF], np.uint8))
+    assert np.isnan(v).all()
+    assert fp8.encode_e4m3(np.array([np.nan]))[0] & 0x7F == 0x7F
+
+
+def test_every_finite_code_round_trips():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    assert np.array_equal(fp8.encode_e4m3(fp8.decode_e4m3(codes)), codes)
+
+
+def test_encode_matches_torch_on_random_in_range_values():
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1.0, 30.0, 120.0)])
+    x = x[np.abs(x) < 440].astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(fp8.encode_e4m3(x), want)
+
+
+def test_ties_round_to_even_and_saturation():
+    enc = lambda v: int(fp8.encode_e4m3(np.array([v]))[0])
+    assert enc(1.0625) == 0x38      # halfway 1.0 / 1.125 -> even mantissa 0
+    assert enc(1.1875) == 0x3A      # halfway 1.125 / 1.25 -> even mantissa 2
+    assert enc(2.0 ** -10) == 0x00  # halfway 0 / 2^-9 -> 0
+    assert enc(3 * 2.0 ** -10) == 0x02
+    assert enc(15 * 2.0 ** -10) == 0x08  # halfway 7*2^-9 / 2^-6 -> 2^-6 (even)
+    assert enc(1.96875) == 0x40     # halfway 1.875 / 2.0 -> carry into the exponent
+    for v in (448.0, 460.0, 470.0, 1e9):
+        assert enc(v) == 0x7E and enc(-v) == 0xFE
+    assert enc(-0.0) == 0x80 and enc(-2.0 ** -12) == 0x80
+
+
+def test_quantize_scaling_steps():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(4096).astype(np.float32)
+    codes, ds = fp8.quantize_e4m3(x)
+    amax = np.abs(x).max()
+    assert ds == np.float32(amax / np.float32(448.0))
+    i = int(np.argmax(np.abs(x)))
+    assert codes[i] in (0x7E, 0xFE)                         # amax -> +-448
+    # error bound of round-to-nearest: half a step of the code's binade
+    y = x.astype(np.float64) * float(np.float32(448.0) / np.float32(amax))
+    err = np.abs(fp8.decode_e4m3(codes) - y)
+    assert (err <= np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6)).all()
+    # a shared amax larger than the tensor's own
+    codes2, ds2 = fp8.quantize_e4m3(x, amax=2 * amax)
+    assert ds2 == np.float32(np.float32(2 * amax) / np.float32(448.0))
+    assert np.abs(fp8.decode_e4m3(codes2)).max() <= 224.0 + 16
+    z, dz = fp8.quantize_e4m3(np.zeros(7, np.float32))
+    assert (z == 0).all() and dz == 1.0
+
+
+def _brute_attention(parent, seg, past, q, k, v, pk, pv, scale):
+    """Each node's isolated sequence written out by walking parents (one
+    request), then plain softmax attention per (token, head) in fp64."""
+    starts = np.concatenate([[0], np.cumsum(seg)])
+    T, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    out = np.zeros((T, Hq, d))
+    for n in range(len(seg)):
+        chain = []
+        a = n
+        while a >= 0:
+            chain.append(a)
+            a = parent[a]
+        chain.reverse()
+        for t in range(starts[n], starts[n + 1]):
+            keys = [("p", i) for i in range(past)]
+            for a in chain:
+                hi = starts[a + 1] if a != n else t + 1
+                keys += [("s", j) for j in range(starts[a], hi)]
+            for h in range(Hq):
+                kv = h // G
+                kk = np.array([(pk if s == "p" else k)[j, kv] for s, j in keys])
+                vv = np.array([(pv if s == "p" else v)[j, kv] for s, j in keys])
+                s = kk @ q[t, h] * scale
+                w = np.exp(s - s.max())
+                out[t, h] = w @ vv / w.sum()
+    return out
+
+
+def test_attention_fp8_equals_brute_force_on_dequantized_inputs():
+    rng = np.random.default_rng(9)
+    parent, seg, past = [-1, 0, 0, 1], [5, 3, 2, 4], 3
+    T, Hq, Hkv, d = sum(seg), 4, 2, 8
+    raw = {n: rng.standard_normal(s).astype(np.float32) * m for n, s, m in [
+        ("q", (T, Hq, d), 1.0), ("k", (T, Hkv, d), 2.0), ("v", (T, Hkv, d), 0.5),
+        ("pk", (past, Hkv, d), 2.0), ("pv", (past, Hkv, d), 0.5)]}
+    q8, sq = fp8.quantize_e4m3(raw["q"])
+    ak = max(np.abs(raw["k"]).max(), np.abs(raw["pk"]).max())
+    av = max(np.abs(raw["v"]).max(), np.abs(raw["pv"]).max())
+    k8, sk = fp8.quantize_e4m3(raw["k"], ak)
+    pk8, _ = fp8.quantize_e4m3(raw["pk"], ak)
+    v8, sv = fp8.quantize_e4m3(raw["v"], av)
+    pv8, _ = fp8.quantize_e4m3(raw["pv"], av)
+    deq = lambda c, s: fp8.decode_e4m3(c) * float(s)
+    scale = 1 / math.sqrt(d)
+    want = _brute_attention(parent, seg, past, deq(q8, sq), deq(k8, sk), deq(v8, sv),
+                            deq(pk8, sk), deq(pv8, sv), scale)
+    tree = ([0, 4], parent, seg, [past])
+    got = fp8.attention_fp8(tree, q8, k8, v8, pk8, pv8, (sq, sk, sv), scale)
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
+    # the (token, head) form agrees with the full form
+    rows = np.array([[0, 0], [T - 1, 3], [6, 1]])
+    part = fp8.attention_fp8(tree, q8, k8, v8, pk8, pv8, (sq, sk, sv), scale, rows)
+    np.testing.assert_allclose(part, got[rows[:, 0], rows[:, 1]], rtol=0, atol=0)
