@@ -56,6 +56,7 @@ extern "C" {
 /* ---- element types ----------------------------------------------------- */
 #define FLIDE_F32 0
 #define FLIDE_BF16 1
+#define FLIDE_E4M3 2 /* 8-bit e4m3 codes (flide_fork_attn_fp8, flide_quantize_e4m3) */
 
 /* ---- flags for flide_fork_attn / flide_fork_gdn ------------------------ */
 #define FLIDE_FLAG_PORTABLE 1 /* force the portable SIMT kernels (any d, any dtype) */
@@ -168,6 +169,50 @@ int flide_fork_attn(const void *q, const void *k, const void *v,
                     flide_tree_index *idx, int32_t Hq, int32_t Hkv, int32_t d,
                     int32_t dtype, float scale, void *out, int32_t flags,
                     flide_stream stream);
+
+/*
+ * Fork attention over e4m3 inputs (the pages run Flide in FP8 where the
+ * hardware has it: techfi24.com, "Exact State Forking" and "Performances").
+ * Same keys and arguments as flide_fork_attn, with
+ *   q [T, Hq, 128], k, v [T, Hkv, 128], past_k, past_v [past_rows, Hkv, 128]
+ *          e4m3 codes (one byte each, as written by flide_quantize_e4m3)
+ *   descale  device float[3] = {sq, sk, sv}: the values are sq*q, sk*k,
+ *          sv*v; past rows use sk and sv (quantise past and new rows with one
+ *          shared amax, see flide_amax)
+ *   out    [T, Hq, 128] bf16
+ * computes o = softmax(scale * (sq q)(sk k)^T)(sv v) with fp32 accumulation.
+ * Tensor-core kernel (kind::f8f6f4) only: d == 128, 128 % (Hq/Hkv) == 0 and
+ * idx->max_depth <= 8, else FLIDE_ERR_SHAPE.  The softmax weights are rounded
+ * to e4m3 (relative error <= 2^-4, absolute <= 2^-16 of the row's largest
+ * weight) before they multiply v; the row sums use the unrounded weights.
+ * Uses idx->work as scratch.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA.
+ */
+int flide_fork_attn_fp8(const void *q, const void *k, const void *v,
+                        const void *past_k, const void *past_v, int32_t past_rows,
+                        flide_tree_index *idx, int32_t Hq, int32_t Hkv, int32_t d,
+                        const float *descale, float scale, void *out,
+                        flide_stream stream);
+
+/*
+ * Absolute maximum for per-tensor e4m3 scaling.  *amax (device float) becomes
+ * max(|x_i|) over the n elements of x (FLIDE_F32 or FLIDE_BF16, 16-byte
+ * aligned), or max(*amax, that) when `accumulate` is non-zero, so several
+ * tensors (past and new K rows, say) can share one scale.  NaN entries are
+ * ignored.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA.
+ */
+int flide_amax(const void *x, int64_t n, int32_t dtype, float *amax, int32_t accumulate,
+               flide_stream stream);
+
+/*
+ * Per-tensor e4m3 quantisation: with a = *amax (device float), inv = 448 / a
+ * and out[i] = e4m3(x[i] * inv), both float32 operations rounded to nearest
+ * and the code rounded to nearest even, magnitudes above 448 saturating to
+ * 448; *descale (device float, may be NULL) = a / 448.  a == 0 gives inv =
+ * descale = 1.  x: n elements of FLIDE_F32 or FLIDE_BF16, 16-byte aligned;
+ * out: n bytes, 8-byte aligned.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA.
+ */
+int flide_quantize_e4m3(const void *x, int64_t n, int32_t dtype, const float *amax,
+                        uint8_t *out, float *descale, flide_stream stream);
 
 /*
  * Fork attention without caller-provided scratch.  (No counterpart in the

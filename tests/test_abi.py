@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "flide.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(flide_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(flide_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exists_and_loads():

@@ -14,8 +14,8 @@ int fork_attn_portable(const void *q, const void *k, const void *v, const void *
                        int dtype, float scale, void *out, cudaStream_t s);
 bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, int dtype);
 int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, const void *pv,
-                 int past_rows, const flide_tree_index *x, int Hq, int Hkv, float scale,
-                 void *out, cudaStream_t s);
+                 int past_rows, const flide_tree_index *x, int Hq, int Hkv, int dtype,
+                 const float *descale, float scale, void *out, cudaStream_t s);
 bool fork_gdn_tc_supported(int dk, int dv, int dtype);
 int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
                 const float *state_in, const flide_tree_index *x, int H, void *out,
@@ -125,11 +125,25 @@ int flide_fork_attn(const void *q, const void *k, const void *v, const void *pas
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || past_rows < 0) return FLIDE_ERR_SHAPE;
   if ((past_k == nullptr) != (past_v == nullptr)) return FLIDE_ERR_SHAPE;
   if (past_k == nullptr) past_rows = 0;
+  if (dtype == FLIDE_E4M3) return FLIDE_ERR_SHAPE;  // needs descale factors: flide_fork_attn_fp8
   if (!(flags & FLIDE_FLAG_PORTABLE) && fork_attn_tc_supported(idx, Hq, Hkv, d, dtype))
-    return fork_attn_tc(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, scale, out,
-                        (cudaStream_t)stream);
+    return fork_attn_tc(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, dtype, nullptr, scale,
+                        out, (cudaStream_t)stream);
   return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,
                             (cudaStream_t)stream);
+}
+
+int flide_fork_attn_fp8(const void *q, const void *k, const void *v, const void *past_k,
+                        const void *past_v, int32_t past_rows, flide_tree_index *idx, int32_t Hq,
+                        int32_t Hkv, int32_t d, const float *descale, float scale, void *out,
+                        flide_stream stream) {
+  if (!idx || !q || !k || !v || !out || !descale) return FLIDE_ERR_SHAPE;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || past_rows < 0) return FLIDE_ERR_SHAPE;
+  if ((past_k == nullptr) != (past_v == nullptr)) return FLIDE_ERR_SHAPE;
+  if (past_k == nullptr) past_rows = 0;
+  if (!fork_attn_tc_supported(idx, Hq, Hkv, d, FLIDE_E4M3)) return FLIDE_ERR_SHAPE;
+  return fork_attn_tc(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, FLIDE_E4M3, descale,
+                      scale, out, (cudaStream_t)stream);
 }
 
 int flide_fork_gdn(const void *q, const void *k, const void *v, const float *g,

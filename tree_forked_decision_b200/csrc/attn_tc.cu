@@ -1,5 +1,5 @@
 // attn_tc.cu -- fork attention on the 5th-generation tensor cores (sm_100a):
-// bf16 q/k/v, head dim 128, fp32 accumulation and online softmax.
+// bf16 or e4m3 q/k/v, head dim 128, fp32 accumulation and online softmax.
 //
 // What it computes (kongchang.com article on Flide, "ForkAttention" and
 // attention-mask sections): every query token attends to exactly the keys of
@@ -44,6 +44,16 @@
 // [256h+128, 256h+256) for O.
 // Every wait is bounded; on expiry the CTA records FLIDE_ERR_TIMEOUT, drains
 // its in-flight copies and MMAs, frees TMEM and exits.
+//
+// e4m3 variant (F8 = true): q, k, v and the past rows are e4m3 codes with one
+// descale factor per tensor (q, k, v; past rows share k's and v's).  A 128-dim
+// row is one 128-byte swizzle row, so Q, K and V tiles are half the bytes;
+// S = Q K^T and O += P V run as kind::f8f6f4 MMAs (K = 32 per instruction).
+// P is written to TMEM as e4m3, four keys per column, scaled by 2^6: the O
+// rescale threshold is 2^2 instead of 2^8, so p <= 4 and 2^6 p <= 256 stays
+// below the format's largest value 448, and weights down to 2^-12 keep a
+// normal e4m3 code.  The row sum uses the unrounded p; the descale factors of
+// q and k fold into the softmax scale and v's into the final normalisation.
 #include <cstddef>
 
 #include "common.cuh"
@@ -106,6 +116,7 @@ struct Misc {
 struct TcParams {
   flide_tree_index x;
   __nv_bfloat16 *out;
+  const float *descale;            // e4m3 inputs: {q, k, v} descale factors
   int Hq, Hkv, G, mtok, has_past;  // mtok = tokens per 128-row half
   float qk_log2;                   // scale * log2(e)
 };
@@ -234,6 +245,7 @@ __device__ __forceinline__ void tile_at(const Misc &ms, int j, Span &sp, int &of
   off = (j - sp.tile0) * BN;
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_pk,
@@ -246,6 +258,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const flide_tree_index &x = p.x;
   auto bar = [&](int i) -> uint32_t { return sb + SM_BAR + 8 * i; };
+  constexpr int kEsz = F8 ? 1 : 2;    // bytes per element
+  constexpr int kSlabs = F8 ? 1 : 2;  // 128-byte swizzle slabs per 128-dim row
 
   if (warp == 8) {
     if (lane == 0) {
@@ -273,9 +287,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(bar(B_Q), 2 * BM * 128 * 2);
+        mbar_arrive_expect_tx(bar(B_Q), 2 * BM * 128 * kEsz);
         for (int h = 0; h < 2; ++h)
-          for (int s = 0; s < 2; ++s)
+          for (int s = 0; s < kSlabs; ++s)
             tma_load_3d(sb + SM_Q + h * 32768 + s * 16384, &tm_q, bar(B_Q), 64 * s, hk * p.G,
                         t0 + h * p.mtok);
         int jk = 0, jv = 0;  // tiles issued
@@ -292,17 +306,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(B_K_FULL + st), BN * 128 * 2);
+          mbar_arrive_expect_tx(bar(B_K_FULL + st), BN * 128 * kEsz);
           tma_load_3d(sb + SM_K + st * 32768, mk, bar(B_K_FULL + st), 0, hk, row);
-          tma_load_3d(sb + SM_K + st * 32768 + 16384, mk, bar(B_K_FULL + st), 64, hk, row);
+          if (!F8) tma_load_3d(sb + SM_K + st * 32768 + 16384, mk, bar(B_K_FULL + st), 64, hk, row);
           ++jk;
           if (j >= 2 && !mbar_wait(bar(B_V_FREE + st), ((j >> 1) - 1) & 1, abort_flag, kTimeoutNs)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(B_V_FULL + st), BN * 128 * 2);
+          mbar_arrive_expect_tx(bar(B_V_FULL + st), BN * 128 * kEsz);
           tma_load_3d(sb + SM_V + st * 32768, mv, bar(B_V_FULL + st), 0, hk, row);
-          tma_load_3d(sb + SM_V + st * 32768 + 16384, mv, bar(B_V_FULL + st), 64, hk, row);
+          if (!F8) tma_load_3d(sb + SM_V + st * 32768 + 16384, mv, bar(B_V_FULL + st), 64, hk, row);
           ++jv;
         }
         if (!ok) {
@@ -317,22 +331,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp == 9) {
       // ------------------------------------------------------------ MMA
       if (lane == 0) {
-        constexpr uint32_t id_s = idesc_bf16(BM, BN, false);
-        constexpr uint32_t id_pv = idesc_bf16(BM, 128, true);
+        constexpr uint32_t id_s = F8 ? idesc_e4m3(BM, BN, false) : idesc_bf16(BM, BN, false);
+        constexpr uint32_t id_pv = F8 ? idesc_e4m3(BM, 128, true) : idesc_bf16(BM, 128, true);
+        // one instruction covers 32 bytes of K: 16 bf16 or 32 e4m3 elements;
+        // in both cases 8 TMEM columns of P and 32 bytes of a K-major row
         auto qk = [&](int h, int st) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < 4 * kSlabs; ++kk) {
             const uint64_t a = sdesc_sw128(sb + SM_Q + h * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
             const uint64_t b = sdesc_sw128(sb + SM_K + st * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            mma_bf16(tmem + h * 256, a, b, id_s, kk > 0 ? 1u : 0u);
+            if (F8) mma_f8(tmem + h * 256, a, b, id_s, kk > 0 ? 1u : 0u);
+            else mma_bf16(tmem + h * 256, a, b, id_s, kk > 0 ? 1u : 0u);
           }
         };
         auto pv = [&](int h, int st, bool acc) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t b = sdesc_sw128(sb + SM_V + st * 32768 + kk * 2048, 16384, 1024);
-            mma_bf16_ts(tmem + h * 256 + 128, tmem + h * 256 + kk * 8, b, id_pv,
-                        (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4 * kSlabs; ++kk) {
+            // V is MN-major: one 128-byte row per key, K advances by keys
+            const uint64_t b = sdesc_sw128(sb + SM_V + st * 32768 + kk * (F8 ? 4096 : 2048), 16384, 1024);
+            if (F8)
+              mma_f8_ts(tmem + h * 256 + 128, tmem + h * 256 + kk * 8, b, id_pv, (acc || kk > 0) ? 1u : 0u);
+            else
+              mma_bf16_ts(tmem + h * 256 + 128, tmem + h * 256 + kk * 8, b, id_pv,
+                          (acc || kk > 0) ? 1u : 0u);
           }
         };
         bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kTimeoutNs) &&
@@ -385,7 +406,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int row_anc = valid_row ? x.anc_ptr[row_node] : 0;
       const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's lanes
       const uint32_t t_s = tl + h * 256, t_o = tl + h * 256 + 128;
-      const float c = p.qk_log2;
+      const float c = F8 ? p.qk_log2 * p.descale[0] * p.descale[1] : p.qk_log2;
+      constexpr float kThreshold = F8 ? 2.0f : kRescaleThreshold;
+      constexpr float kPShift = F8 ? 6.0f : 0.0f;  // P stored as 2^kPShift p
       float m_used = -INFINITY, l = 0.f;
       int span_tile0 = -1, vis_lo = 0, vis_hi = 0;
       bool ok = true;
@@ -452,7 +475,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           m_used = mt;
         } else {
           // PV(j-1) of this half is complete (it precedes S(j) in issue order)
-          const bool need = mt > m_used + kRescaleThreshold;
+          const bool need = mt > m_used + kThreshold;
           if (__any_sync(0xffffffffu, need)) {
             const float f = need ? exp2f(m_used - mt) : 1.f;
 #pragma unroll 1
@@ -467,20 +490,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (need) m_used = mt;
           }
         }
-        const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+        const float m_sub = ((m_used == -INFINITY) ? 0.f : m_used) - kPShift;
         // p = 2^(s*c - m): paired scale-and-shift, SFU exp2, paired row-sum
         // chains; P packed to bf16x2 in place into sr[0..63]
         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_sub, -m_sub);
         uint64_t acc[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[k] = 0ull;
+        if (F8) {
+          // P as e4m3 codes, four keys per word, into sr[0..31]
 #pragma unroll
-        for (int i = 0; i < BN; i += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2), x0, x1);
-          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-          acc[(i >> 1) & 3] = f2_add(acc[(i >> 1) & 3], f2_pack(e0, e1));
-          sr[i >> 1] = pack_bf16x2(e0, e1);
+          for (int i = 0; i < BN; i += 4) {
+            float x0, x1, x2, x3;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2), x0, x1);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])), c2, nm2), x2, x3);
+            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            const float e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+            acc[(i >> 1) & 3] = f2_add(acc[(i >> 1) & 3], f2_pack(e0, e1));
+            acc[((i >> 1) + 1) & 3] = f2_add(acc[((i >> 1) + 1) & 3], f2_pack(e2, e3));
+            sr[i >> 2] = pack_e4m3x4(e0, e1, e2, e3);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < BN; i += 2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2), x0, x1);
+            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            acc[(i >> 1) & 3] = f2_add(acc[(i >> 1) & 3], f2_pack(e0, e1));
+            sr[i >> 1] = pack_bf16x2(e0, e1);
+          }
         }
         {
           float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -490,7 +528,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           f2_unpack(acc[3], d0, d1);
           l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
-        tmem_st64(t_s, *reinterpret_cast<uint32_t(*)[64]>(sr));
+        if (F8) tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        else tmem_st64(t_s, *reinterpret_cast<uint32_t(*)[64]>(sr));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_FULL + h));
@@ -500,7 +539,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         uint32_t orr[128];
         tmem_ld128(t_o, orr);
         if (valid_row) {
-          const float inv = 1.f / l;
+          const float inv = (F8 ? p.descale[2] : 1.f) / l;
           __nv_bfloat16 *o = p.out + ((size_t)t * p.Hq + hk * p.G + g) * 128;
 #pragma unroll
           for (int q8 = 0; q8 < 16; ++q8) {
@@ -544,17 +583,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, heads, 128] bf16 viewed as a 3-D tensor (dim, head, row); box of
-// 64 dims x box_heads heads x box_rows rows, 128-byte swizzle.
+// [rows, heads, 128] bf16 (esz 2) or e4m3 (esz 1) viewed as a 3-D tensor
+// (dim, head, row); box of 128 bytes of dims x box_heads heads x box_rows
+// rows, 128-byte swizzle.
 bool make_map(CUtensorMap *m, const void *base, int heads, long rows, int box_heads,
-              int box_rows) {
+              int box_rows, int esz) {
   EncodeTiledFn enc = encode_fn();
   if (!enc || rows <= 0) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {256, (cuuint64_t)heads * 256};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint64_t strides[2] = {(cuuint64_t)128 * esz, (cuuint64_t)heads * 128 * esz};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+  return enc(m, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(base), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -562,7 +603,7 @@ bool make_map(CUtensorMap *m, const void *base, int heads, long rows, int box_he
 }  // namespace
 
 bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, int dtype) {
-  if (dtype != FLIDE_BF16 || d != 128 || Hkv <= 0 || Hq % Hkv != 0) return false;
+  if ((dtype != FLIDE_BF16 && dtype != FLIDE_E4M3) || d != 128 || Hkv <= 0 || Hq % Hkv != 0) return false;
   const int G = Hq / Hkv;
   if (G > BM || BM % G != 0) return false;
   if (x->max_depth > kMaxLevels) return false;
@@ -570,34 +611,40 @@ bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, i
 }
 
 int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, const void *pv,
-                 int past_rows, const flide_tree_index *x, int Hq, int Hkv, float scale,
-                 void *out, cudaStream_t s) {
+                 int past_rows, const flide_tree_index *x, int Hq, int Hkv, int dtype,
+                 const float *descale, float scale, void *out, cudaStream_t s) {
   const int G = Hq / Hkv;
   const int mtok = BM / G;  // tokens per 128-row half; a tile is 2*mtok tokens
+  const bool f8 = dtype == FLIDE_E4M3;
+  const int esz = f8 ? 1 : 2;
+  if (f8 && descale == nullptr) return FLIDE_ERR_SHAPE;
   CUtensorMap mq, mk, mv, mpk, mpv;
   const long T = x->T > 0 ? x->T : 1;
-  if (!make_map(&mq, q, Hq, T, G, mtok)) return FLIDE_ERR_CUDA;
-  if (!make_map(&mk, k, Hkv, T, 1, BN)) return FLIDE_ERR_CUDA;
-  if (!make_map(&mv, v, Hkv, T, 1, BN)) return FLIDE_ERR_CUDA;
+  if (!make_map(&mq, q, Hq, T, G, mtok, esz)) return FLIDE_ERR_CUDA;
+  if (!make_map(&mk, k, Hkv, T, 1, BN, esz)) return FLIDE_ERR_CUDA;
+  if (!make_map(&mv, v, Hkv, T, 1, BN, esz)) return FLIDE_ERR_CUDA;
   const bool has_past = pk != nullptr && past_rows > 0;
-  if (!make_map(&mpk, has_past ? pk : k, Hkv, has_past ? past_rows : T, 1, BN)) return FLIDE_ERR_CUDA;
-  if (!make_map(&mpv, has_past ? pv : v, Hkv, has_past ? past_rows : T, 1, BN)) return FLIDE_ERR_CUDA;
+  if (!make_map(&mpk, has_past ? pk : k, Hkv, has_past ? past_rows : T, 1, BN, esz)) return FLIDE_ERR_CUDA;
+  if (!make_map(&mpv, has_past ? pv : v, Hkv, has_past ? past_rows : T, 1, BN, esz)) return FLIDE_ERR_CUDA;
 
-  // the shared-memory opt-in is per device; remember it for the first 64
-  static bool attr_set[64] = {};
+  // the shared-memory opt-in is per device and kernel; remember it for the
+  // first 64 devices
+  static bool attr_set[2][64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLIDE_ERR_CUDA;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return FLIDE_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  if (dev < 0 || dev >= 64 || !attr_set[f8][dev]) {
+    const cudaError_t e =
+        f8 ? cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
+           : cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return FLIDE_ERR_CUDA;
+    if (dev >= 0 && dev < 64) attr_set[f8][dev] = true;
   }
   attn_items_kernel<<<1, 1024, 0, s>>>(*x, Hkv, 2 * mtok);
   FLIDE_LAUNCH_CHECK();
   TcParams prm;
   prm.x = *x;
   prm.out = (__nv_bfloat16 *)out;
+  prm.descale = descale;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.G = G;
@@ -607,7 +654,10 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
   const long grid = (long)Hkv * ((x->T + 2 * mtok - 1) / (2 * mtok) + 2L * x->R);
   if (grid <= 0) return FLIDE_OK;
   if (grid > 0x7fffffffL) return FLIDE_ERR_CAPACITY;
-  attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mpk, mpv, prm);
+  if (f8)
+    attn_tc_kernel<true><<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mpk, mpv, prm);
+  else
+    attn_tc_kernel<false><<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mpk, mpv, prm);
   FLIDE_LAUNCH_CHECK();
   return FLIDE_OK;
 }
@@ -662,8 +712,8 @@ extern "C" int flide_fork_attn_noalloc(const void *q, const void *k, const void 
     flide_tree_index x = *idx;  // same index, work table moved to the fixed array
     x.work = work;
     x.work_len = kNoAllocMaxRequests + 1;
-    return fork_attn_tc(q, k, v, past_k, past_v, past_rows, &x, Hq, Hkv, scale, out,
-                        (cudaStream_t)stream);
+    return fork_attn_tc(q, k, v, past_k, past_v, past_rows, &x, Hq, Hkv, dtype, nullptr, scale,
+                        out, (cudaStream_t)stream);
   }
   // the CUDA-core kernel keeps no per-call table
   return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,

@@ -16,7 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libflide.so")
 
 OK, ERR_INVALID, ERR_SHAPE, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT = range(6)
-F32, BF16 = 0, 1
+F32, BF16, E4M3 = 0, 1, 2
 FLAG_PORTABLE = 1
 COUNTS = 16
 CNT = dict(N=0, T=1, PAST=2, DEPTH=3, SLOTS=4, BRANCH_TOK=5, ROOT_TOK=6, CKPT_ROWS=7)
@@ -33,7 +33,7 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_option_probs", "flide_pool_create", "flide_pool_destroy", "flide_pool_append",
            "flide_pool_release", "flide_pool_length", "flide_pool_free_blocks", "flide_pool_export",
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
-           "flide_strerror"]
+           "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -115,6 +115,12 @@ def _lib():
         lib.flide_history_gather.restype = ctypes.c_int
         lib.flide_selftest_wait_timeout.argtypes = [P, I32, I32, P]
         lib.flide_selftest_wait_timeout.restype = ctypes.c_int
+        lib.flide_fork_attn_fp8.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, P, F, P, P]
+        lib.flide_fork_attn_fp8.restype = ctypes.c_int
+        lib.flide_amax.argtypes = [P, ctypes.c_int64, I32, P, I32, P]
+        lib.flide_amax.restype = ctypes.c_int
+        lib.flide_quantize_e4m3.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
+        lib.flide_quantize_e4m3.restype = ctypes.c_int
         lib.flide_strerror.argtypes = [ctypes.c_int32]
         lib.flide_strerror.restype = ctypes.c_char_p
         _LIB = lib
@@ -228,6 +234,59 @@ def fork_attn(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None,
                                   float(scale), _ptr(out), flags, _stream(stream)),
            "flide_fork_attn")
     return out
+
+
+def fork_attn_fp8(q8, k8, v8, index: TreeIndex, scale: float, descale, past_k=None, past_v=None,
+                  out=None, stream=None):
+    """Fork attention over e4m3 codes (uint8 tensors [T, H, 128]); descale is
+    a float32 device tensor [3] = (sq, sk, sv); past rows use sk and sv.
+    Returns bf16 [T, Hq, 128]."""
+    T, Hq, d = q8.shape
+    Hkv = k8.shape[1]
+    for t in (q8, k8, v8, past_k, past_v):
+        if t is not None and (t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_contiguous()):
+            raise TypeError("e4m3 inputs must be contiguous uint8 / float8_e4m3fn tensors")
+    if descale.dtype != torch.float32 or descale.numel() < 3:
+        raise TypeError("descale must be a float32 tensor of 3 entries")
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    past_rows = 0 if past_k is None else past_k.shape[0]
+    if past_rows == 0:
+        past_k = past_v = None
+    _check(_lib().flide_fork_attn_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(past_k), _ptr(past_v),
+                                      past_rows, ctypes.byref(index.c), Hq, Hkv, d, _ptr(descale),
+                                      float(scale), _ptr(out), _stream(stream)),
+           "flide_fork_attn_fp8")
+    return out
+
+
+def amax(x, out=None, accumulate: bool = False, stream=None):
+    """float32 device tensor [1] = max |x| (max with its current value when
+    accumulate), for per-tensor e4m3 scaling."""
+    if not x.is_contiguous():
+        raise TypeError("x must be contiguous")
+    if out is None:
+        out = torch.zeros(1, dtype=torch.float32, device=x.device)
+    _check(_lib().flide_amax(_ptr(x), x.numel(), _dtype_code(x), _ptr(out), int(bool(accumulate)),
+                             _stream(stream)), "flide_amax")
+    return out
+
+
+def quantize_e4m3(x, amax_t=None, out=None, descale=None, stream=None):
+    """e4m3 codes of x (uint8, x's shape) scaled so that amax_t (default: x's
+    own absolute maximum) maps to 448, and the descale factor amax / 448
+    (float32 device tensor [1])."""
+    if not x.is_contiguous():
+        raise TypeError("x must be contiguous")
+    if amax_t is None:
+        amax_t = amax(x, stream=stream)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if descale is None:
+        descale = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(_lib().flide_quantize_e4m3(_ptr(x), x.numel(), _dtype_code(x), _ptr(amax_t), _ptr(out),
+                                      _ptr(descale), _stream(stream)), "flide_quantize_e4m3")
+    return out, descale
 
 
 def fork_attn_noalloc(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None,

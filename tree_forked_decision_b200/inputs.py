@@ -215,6 +215,24 @@ def attn_inputs(tree: Tree, Hq: int, Hkv: int, d: int, dtype: torch.dtype,
                 past_k=_to(pk, dtype), past_v=_to(pv, dtype))
 
 
+def fp8_attn_inputs(tree: Tree, Hq: int, Hkv: int, d: int, rng: np.random.Generator,
+                    amp: float = 64.0):
+    """e4m3 codes (uint8 tensors) of amp * N(0,1) for q [T,Hq,d], k, v [T,Hkv,d]
+    and past_k, past_v [sum(past),Hkv,d], cast by torch's float8_e4m3fn
+    conversion, with descale = (1/amp, 1/amp, 1/amp) (float32 [3]): the
+    decoded values are N(0,1) to within the format's rounding.  amp * 6 stays
+    below the format's largest value 448 for these sample sizes."""
+    T, P = tree.T, tree.P_past
+
+    def codes(shape):
+        x = normals(rng, shape) * np.float32(amp)
+        return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8)
+
+    return dict(q=codes((T, Hq, d)), k=codes((T, Hkv, d)), v=codes((T, Hkv, d)),
+                past_k=codes((P, Hkv, d)), past_v=codes((P, Hkv, d)),
+                descale=torch.full((3,), 1.0 / amp, dtype=torch.float32))
+
+
 def _l2n(x: np.ndarray) -> torch.Tensor:
     """Rows scaled to unit L2 norm, in float32."""
     t = torch.from_numpy(x)
