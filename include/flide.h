@@ -184,7 +184,8 @@ int flide_fork_attn(const void *q, const void *k, const void *v,
  * Tensor-core kernel (kind::f8f6f4) only: d == 128, 128 % (Hq/Hkv) == 0 and
  * idx->max_depth <= 8, else FLIDE_ERR_SHAPE.  The softmax weights are rounded
  * to e4m3 (relative error <= 2^-4, absolute <= 2^-16 of the row's largest
- * weight) before they multiply v; the row sums use the unrounded weights.
+ * weight) before they multiply v; one in eight comes from a polynomial exp2
+ * (relative error < 1e-4); the row sums use the unrounded weights.
  * Uses idx->work as scratch.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA.
  */
 int flide_fork_attn_fp8(const void *q, const void *k, const void *v,

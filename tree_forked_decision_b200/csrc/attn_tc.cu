@@ -52,7 +52,8 @@
 // P is written to TMEM as e4m3, four keys per column, scaled by 2^6: the O
 // rescale threshold is 2^2 instead of 2^8, so p <= 4 and 2^6 p <= 256 stays
 // below the format's largest value 448, and weights down to 2^-12 keep a
-// normal e4m3 code.  The row sum uses the unrounded p; the descale factors of
+// normal e4m3 code.  One exponential pair in eight is evaluated on the FMA
+// pipe (ex2_poly2).  The row sum uses the unrounded p; the descale factors of
 // q and k fold into the softmax scale and v's into the final normalisation.
 #include <cstddef>
 
@@ -504,7 +505,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             float x0, x1, x2, x3;
             f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2), x0, x1);
             f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])), c2, nm2), x2, x3);
-            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            // one pair in eight on the FMA pipe: the special-function unit's
+            // exp2 throughput bounds this loop once the MMAs take e4m3
+            float e0, e1;
+            if ((i >> 2) % 4 == 0) {
+              f2_unpack(ex2_poly2(x0, x1), e0, e1);
+            } else {
+              e0 = ex2_approx(x0);
+              e1 = ex2_approx(x1);
+            }
             const float e2 = ex2_approx(x2), e3 = ex2_approx(x3);
             acc[(i >> 1) & 3] = f2_add(acc[(i >> 1) & 3], f2_pack(e0, e1));
             acc[((i >> 1) + 1) & 3] = f2_add(acc[((i >> 1) + 1) & 3], f2_pack(e2, e3));

@@ -214,6 +214,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for a pair of floats on the FMA pipe instead of the special-function
+// unit: x = n + f with n = rint(x) (the 1.5*2^23 shift) and f in [-1/2, 1/2],
+// 2^f by a cubic whose coefficients minimise the maximum relative error on
+// that interval (found by linear programming; 7.5e-5), then n added to the
+// exponent field.  x is clamped at -126 (no subnormal results).
+__device__ __forceinline__ uint64_t ex2_poly2(float x0, float x1) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  uint64_t x, sh, nsh, t, f;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(sh) : "f"(kShift));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(nsh) : "f"(-kShift));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(sh));   // n in the low mantissa bits
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(t), "l"(nsh));  // n as a float
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(f));    // f = x - n
+  uint64_t c3, c2, c1, c0, p;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(0.05517222f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(0.24261115f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c1) : "f"(0.69326085f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c0) : "f"(0.99992806f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
+  const uint32_t n0 = (uint32_t)t, n1 = (uint32_t)(t >> 32);
+  const uint32_t r0 = (uint32_t)p + (n0 << 23), r1 = (uint32_t)(p >> 32) + (n1 << 23);
+  return (uint64_t)r0 | ((uint64_t)r1 << 32);
+}
+
 // max of three floats (sm_100 three-input form)
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float r;
