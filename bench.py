@@ -683,6 +683,42 @@ def main():
                    "frac_of_hbm_peak": hbytes / (h_ms / 1000.0) / 1e9 / hbm,
                    "note": "resume of every request's history (roots of this step) from the block pool "
                            "into packed past K/V and GDN state_in"}
+        # the resumed batch (branch tokens only, past = the histories) with its
+        # attention reading the past in place from the blocks, against the same
+        # attention over the packed copy
+        tree_w, keep = inputs.warm_variant(tree)
+        if tree_w.P_past == rows and a["d"] == 128 and step.q.dtype == torch.bfloat16:
+            ridx = torch.from_numpy(keep).to(device)
+            qw, kw, vw = (t[ridx].contiguous() for t in (step.q, step.k, step.v))
+            dtw = flide.DeviceTree(*tree_w.arrays(), max_depth=max(tree_w.levels, 1), device=device)
+            idxw = flide.TreeIndex(dtw.R, dtw.N, dtw.T, dtw.max_depth, device=device)
+            flide.tree_build(dtw, idxw)
+            _, pkw, pvw, _ = store.resume(slots)
+            ow1 = torch.empty_like(qw)
+            ow2 = torch.empty_like(qw)
+            pk_run = lambda: flide.fork_attn(qw, kw, vw, idxw, step.scale, past_k=pkw, past_v=pvw, out=ow1)
+            pg_run = lambda: store.fork_attn_paged(qw, kw, vw, idxw, step.scale, slots, out=ow2)
+            for _ in range(max(args.warmup, 1)):
+                pk_run()
+                pg_run()
+            pev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+            barrier()
+            for i in range(args.steps):
+                pev[i][0].record()
+                pk_run()
+                pev[i][1].record()
+                pg_run()
+                pev[i][2].record()
+            torch.cuda.synchronize()
+            barrier()
+            if idxw.status() != 0:
+                raise SystemExit(f"device status {idxw.status()} in the paged attention")
+            history.update(
+                packed_attn_ms=max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in pev), pg, device),
+                paged_attn_ms=max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in pev), pg, device),
+                paged_equals_packed=bool(torch.equal(ow1, ow2)),
+                paged_note="resumed batch: attention over the packed copy vs past read in place from "
+                           "the blocks (flide_fork_attn_paged, no gather)")
         del store
 
     # e4m3 fork attention on the same tree and values: q, k, v and the past

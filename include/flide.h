@@ -195,6 +195,34 @@ int flide_fork_attn_fp8(const void *q, const void *k, const void *v,
                         flide_stream stream);
 
 /*
+ * Fork attention with the past rows read in place from a block-paged history
+ * pool (the pool of flide_pool_* / flide_history_*), with no packed copy:
+ * request r's past rows are history rows 0 .. past_len[r]-1 (past_len as
+ * given to flide_tree_build) of slot req_slot[r], history row i stored at
+ * pool row block_table[req_slot[r] * max_blocks + i / block_rows] *
+ * block_rows + i % block_rows.  (The pages resume from a saved prefix and
+ * grow it step by step -- kongchang.com closing section; techfi24.com,
+ * "Exact State Forking" -- the paged layout is this library's.)
+ *   pool_k, pool_v [n_blocks * block_rows, Hkv, 128] dtype
+ *   block_table    device int32 [n_slots * max_blocks]
+ *   req_slot       device int32 [idx->R]; a request with past rows needs
+ *                  0 <= slot < n_slots and past_len <= max_blocks * block_rows
+ *   block_rows     a multiple of 128 (one key tile never spans two blocks)
+ * Otherwise as flide_fork_attn (dtype FLIDE_BF16) or flide_fork_attn_fp8
+ * (dtype FLIDE_E4M3, with descale; the pool holds e4m3 codes); tensor-core
+ * kernel only.  Device errors: FLIDE_ERR_INVALID in idx->status for a bad
+ * slot, a history longer than the slot's table or a table entry outside
+ * [0, n_blocks) (block 0 is read in its place).  Host errors:
+ * FLIDE_ERR_SHAPE, FLIDE_ERR_CAPACITY, FLIDE_ERR_CUDA.
+ */
+int flide_fork_attn_paged(const void *q, const void *k, const void *v, const void *pool_k,
+                          const void *pool_v, int32_t n_blocks, int32_t block_rows,
+                          const int32_t *block_table, int32_t max_blocks, const int32_t *req_slot,
+                          int32_t n_slots, flide_tree_index *idx, int32_t Hq, int32_t Hkv,
+                          int32_t d, int32_t dtype, const float *descale, float scale, void *out,
+                          flide_stream stream);
+
+/*
  * Absolute maximum for per-tensor e4m3 scaling.  *amax (device float) becomes
  * max(|x_i|) over the n elements of x (FLIDE_F32 or FLIDE_BF16, 16-byte
  * aligned), or max(*amax, that) when `accumulate` is non-zero, so several
@@ -393,6 +421,10 @@ int flide_history_append(const flide_tree_index *idx, const int32_t *req_slot,
  * a request with no history) writes past_len[r] = hist_len[slot], the
  * histories' rows packed in request order into past_k/past_v [past_rows, Hkv, d]
  * and state_in[r] = pool_S[slot] (zeros for -1) when state_in is given.
+ * With past_k = past_v = NULL and past_rows = 0 only past_len (and state_in)
+ * are written: the lengths flide_tree_build needs before flide_fork_attn_paged
+ * reads the rows in place.  dtype FLIDE_F32, FLIDE_BF16 or FLIDE_E4M3 (rows
+ * are copied as bytes).
  * Device errors to *status: FLIDE_ERR_CAPACITY when the rows exceed
  * past_rows, FLIDE_ERR_INVALID for a slot >= max_requests or a row without a
  * block.  R <= 4096. */

@@ -198,3 +198,18 @@ def test_fork_attn_fp8_rejects_unsupported():
     assert lib.flide_fork_attn(flide._ptr(q), flide._ptr(k), flide._ptr(v), None, None, 0,
                                ctypes.byref(idx.c), 4, 2, 128, flide.E4M3, 1.0, flide._ptr(out),
                                0, flide._stream()) == flide.ERR_SHAPE
+
+
+@pytest.mark.parametrize("name", ["attn_fanout_bf16", "mixed_hybrid_bf16", "large_fanout_bf16"])
+def test_fullsize_fork_attn_fp8_sampled(name):
+    """The benched workloads' trees and head counts with e4m3 inputs, checked
+    on the full-size test's row sample (first and last root rows, every
+    branch row of query head 0, random rows) under the same bound."""
+    from test_gpu_fullsize import _rows
+    tree, spec, _, _, rng = inputs.workload(name)
+    a = inputs.fp8_attn_inputs(tree, spec["Hq"], spec["Hkv"], spec["d"], rng)
+    _, idx = build(tree)
+    got, scale = _run_fp8(tree, a, idx)
+    rows = _rows(tree, spec["Hq"], 1500, np.random.default_rng(1))
+    want, tol = _oracle_and_bound(tree, a, scale, rows)
+    _assert_within(got[rows[:, 0], rows[:, 1]], want, tol)

@@ -4,7 +4,9 @@ observation (its root) and scores new options; afterwards the observation and
 the root's end state are appended.  Every step's outputs (attention and GDN,
 observation and option rows) must equal the oracle run from scratch over the
 whole history (resume equals scratch, step after step).  One request ends its
-episode after step 1 and starts a new one in the same slot."""
+episode after step 1 and starts a new one in the same slot.  With blocks of
+128 rows the attention also runs with the past read in place from the blocks
+(flide_fork_attn_paged) and must equal the gathered-past result bit for bit."""
 import math
 
 import numpy as np
@@ -35,11 +37,13 @@ def _cat(chunks):
     return {key: torch.cat([c[key] for c in chunks]) for key in chunks[0]}
 
 
-def test_agent_episode_through_paged_history():
+@pytest.mark.parametrize("block_rows", [16, 128])
+def test_agent_episode_through_paged_history(block_rows):
     rng = np.random.default_rng(21)
     R, steps = 3, 3
-    store = HistoryStore(n_blocks=64, block_rows=16, max_requests=4, max_blocks=16, Hkv=Hkv, d=d,
-                         H=H, dk=dk, dv=dv)
+    n_blocks = 64 if block_rows == 16 else 12
+    store = HistoryStore(n_blocks=n_blocks, block_rows=block_rows, max_requests=4,
+                         max_blocks=16 if block_rows == 16 else 4, Hkv=Hkv, d=d, H=H, dk=dk, dv=dv)
     slots = [0, 1, 2]
     history = [[] for _ in range(R)]  # observation chunks of the current episode
     for step in range(steps):
@@ -64,6 +68,14 @@ def test_agent_episode_through_paged_history():
         has_past = sum(hist_len) > 0
         o = flide.fork_attn(dev["q"], dev["k"], dev["v"], idx, 1 / math.sqrt(d),
                             past_k=pk if has_past else None, past_v=pv if has_past else None)
+        if block_rows % 128 == 0:
+            # same lengths without the packed copy, past rows read in place
+            plen2, state2 = store.resume_lengths([-1 if f else s for f, s in zip(fresh, slots)])
+            o_paged = store.fork_attn_paged(dev["q"], dev["k"], dev["v"], idx, 1 / math.sqrt(d),
+                                            [-1 if f else s for f, s in zip(fresh, slots)])
+            torch.cuda.synchronize()
+            assert torch.equal(plen2, past_len) and torch.equal(state2, state_in)
+            assert torch.equal(o_paged, o)
         node_state = torch.zeros((max(flide.state_slots(tree), 1), H, dv, dk), device="cuda")
         go = flide.fork_gdn(dev["gq"], dev["gk"], dev["gv"], dev["gg"], dev["gb"], idx, node_state,
                             state_in=state_in if has_past else None)
@@ -93,4 +105,4 @@ def test_agent_episode_through_paged_history():
                             f(sdata["gg"]), f(sdata["gb"]))
         assert_close(o.float().cpu().numpy(), want_a[rows], torch.bfloat16)
         assert_close(go.float().cpu().numpy(), want_g[rows], torch.bfloat16)
-    assert store.free_blocks() == 64 - sum(-(-store.length(s) // 16) for s in slots)
+    assert store.free_blocks() == n_blocks - sum(-(-store.length(s) // block_rows) for s in slots)

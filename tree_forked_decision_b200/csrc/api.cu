@@ -15,7 +15,8 @@ int fork_attn_portable(const void *q, const void *k, const void *v, const void *
 bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, int dtype);
 int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, const void *pv,
                  int past_rows, const flide_tree_index *x, int Hq, int Hkv, int dtype,
-                 const float *descale, float scale, void *out, cudaStream_t s);
+                 const float *descale, float scale, void *out, cudaStream_t s,
+                 const PagedPast *paged);
 bool fork_gdn_tc_supported(int dk, int dv, int dtype);
 int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
                 const float *state_in, const flide_tree_index *x, int H, void *out,
@@ -128,7 +129,7 @@ int flide_fork_attn(const void *q, const void *k, const void *v, const void *pas
   if (dtype == FLIDE_E4M3) return FLIDE_ERR_SHAPE;  // needs descale factors: flide_fork_attn_fp8
   if (!(flags & FLIDE_FLAG_PORTABLE) && fork_attn_tc_supported(idx, Hq, Hkv, d, dtype))
     return fork_attn_tc(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, dtype, nullptr, scale,
-                        out, (cudaStream_t)stream);
+                        out, (cudaStream_t)stream, nullptr);
   return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,
                             (cudaStream_t)stream);
 }
@@ -143,7 +144,27 @@ int flide_fork_attn_fp8(const void *q, const void *k, const void *v, const void 
   if (past_k == nullptr) past_rows = 0;
   if (!fork_attn_tc_supported(idx, Hq, Hkv, d, FLIDE_E4M3)) return FLIDE_ERR_SHAPE;
   return fork_attn_tc(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, FLIDE_E4M3, descale,
-                      scale, out, (cudaStream_t)stream);
+                      scale, out, (cudaStream_t)stream, nullptr);
+}
+
+int flide_fork_attn_paged(const void *q, const void *k, const void *v, const void *pool_k,
+                          const void *pool_v, int32_t n_blocks, int32_t block_rows,
+                          const int32_t *block_table, int32_t max_blocks, const int32_t *req_slot,
+                          int32_t n_slots, flide_tree_index *idx, int32_t Hq, int32_t Hkv,
+                          int32_t d, int32_t dtype, const float *descale, float scale, void *out,
+                          flide_stream stream) {
+  if (!idx || !q || !k || !v || !out || !pool_k || !pool_v || !block_table || !req_slot)
+    return FLIDE_ERR_SHAPE;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return FLIDE_ERR_SHAPE;
+  if (n_blocks <= 0 || max_blocks <= 0 || n_slots <= 0 || block_rows <= 0 || block_rows % 128)
+    return FLIDE_ERR_SHAPE;
+  if ((int64_t)n_blocks * block_rows > 0x7fffffffLL) return FLIDE_ERR_CAPACITY;
+  if (dtype == FLIDE_E4M3 && !descale) return FLIDE_ERR_SHAPE;
+  if (!fork_attn_tc_supported(idx, Hq, Hkv, d, dtype)) return FLIDE_ERR_SHAPE;
+  const PagedPast pp{block_table, req_slot, max_blocks, block_rows, n_blocks, n_slots};
+  return fork_attn_tc(q, k, v, pool_k, pool_v, n_blocks * block_rows, idx, Hq, Hkv, dtype,
+                      dtype == FLIDE_E4M3 ? descale : nullptr, scale, out, (cudaStream_t)stream,
+                      &pp);
 }
 
 int flide_fork_gdn(const void *q, const void *k, const void *v, const float *g,

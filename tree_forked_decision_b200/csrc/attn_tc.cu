@@ -111,6 +111,7 @@ struct Misc {
   int valid;
   int n_spans, n_tiles;
   int r, hk, t0, ntok;
+  int slot;  // paged past: the request's history slot
   Span spans[kMaxSpans];
 };
 
@@ -118,6 +119,11 @@ struct TcParams {
   flide_tree_index x;
   __nv_bfloat16 *out;
   const float *descale;            // e4m3 inputs: {q, k, v} descale factors
+  // paged past (block_table != nullptr): history row i of request r is pool
+  // row block_table[req_slot[r] * max_blocks + i / block_rows] * block_rows +
+  // i % block_rows; block_rows is a multiple of the key tile
+  const int32_t *block_table, *req_slot;
+  int max_blocks, block_rows, n_blocks, n_slots;
   int Hq, Hkv, G, mtok, has_past;  // mtok = tokens per 128-row half
   float qk_log2;                   // scale * log2(e)
 };
@@ -199,6 +205,17 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
       return;
     }
     sp[ns++] = Span{SRC_PAST, p0, plen, KIND_FULL, 0, 0};
+    if (p.block_table) {
+      const int slot = p.req_slot[r];
+      if (slot < 0 || slot >= p.n_slots || plen > (long)p.max_blocks * p.block_rows) {
+        if (lane == 0) {
+          set_status(x.status, FLIDE_ERR_INVALID);
+          ms.valid = 0;
+        }
+        return;
+      }
+      if (lane == 0) ms.slot = slot;
+    }
   }
   if (branch) {
     if (br_start > root_start) sp[ns++] = Span{SRC_STREAM, root_start, br_start - root_start, KIND_FULL, 0, 0};
@@ -301,7 +318,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tile_at(ms, j, sp, off);
           const CUtensorMap *mk = sp.src == SRC_PAST ? &tm_pk : &tm_k;
           const CUtensorMap *mv = sp.src == SRC_PAST ? &tm_pv : &tm_v;
-          const int row = sp.start + off;
+          int row = sp.start + off;
+          if (sp.src == SRC_PAST && p.block_table) {
+            // a key tile lies inside one block (block_rows % BN == 0)
+            int b = p.block_table[(size_t)ms.slot * p.max_blocks + off / p.block_rows];
+            if (b < 0 || b >= p.n_blocks) {
+              set_status(x.status, FLIDE_ERR_INVALID);  // no block: read block 0, flag the call
+              b = 0;
+            }
+            row = b * p.block_rows + off % p.block_rows;
+          }
           const int st = j & 1;
           if (j >= 2 && !mbar_wait(bar(B_K_FREE + st), ((j >> 1) - 1) & 1, abort_flag, kTimeoutNs)) {
             ok = false;
@@ -621,7 +647,8 @@ bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, i
 
 int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, const void *pv,
                  int past_rows, const flide_tree_index *x, int Hq, int Hkv, int dtype,
-                 const float *descale, float scale, void *out, cudaStream_t s) {
+                 const float *descale, float scale, void *out, cudaStream_t s,
+                 const PagedPast *paged) {
   const int G = Hq / Hkv;
   const int mtok = BM / G;  // tokens per 128-row half; a tile is 2*mtok tokens
   const bool f8 = dtype == FLIDE_E4M3;
@@ -654,6 +681,12 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
   prm.x = *x;
   prm.out = (__nv_bfloat16 *)out;
   prm.descale = descale;
+  prm.block_table = paged ? paged->block_table : nullptr;
+  prm.req_slot = paged ? paged->req_slot : nullptr;
+  prm.max_blocks = paged ? paged->max_blocks : 0;
+  prm.block_rows = paged ? paged->block_rows : 0;
+  prm.n_blocks = paged ? paged->n_blocks : 0;
+  prm.n_slots = paged ? paged->n_slots : 0;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.G = G;
@@ -722,7 +755,7 @@ extern "C" int flide_fork_attn_noalloc(const void *q, const void *k, const void 
     x.work = work;
     x.work_len = kNoAllocMaxRequests + 1;
     return fork_attn_tc(q, k, v, past_k, past_v, past_rows, &x, Hq, Hkv, dtype, nullptr, scale,
-                        out, (cudaStream_t)stream);
+                        out, (cudaStream_t)stream, nullptr);
   }
   // the CUDA-core kernel keeps no per-call table
   return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,

@@ -9,6 +9,14 @@
 
 namespace flide {
 
+// Past K/V rows read in place from a block-paged history pool: history row i
+// of request r is pool row block_table[req_slot[r] * max_blocks + i /
+// block_rows] * block_rows + i % block_rows.
+struct PagedPast {
+  const int32_t *block_table, *req_slot;
+  int max_blocks, block_rows, n_blocks, n_slots;
+};
+
 // Records the first device-detected error; later ones are dropped.
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
   atomicCAS(status, 0, code);

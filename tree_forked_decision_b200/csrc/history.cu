@@ -133,7 +133,7 @@ __global__ void history_gather_kernel(int R, const int32_t *req_slot, int max_re
   }
   if (threadIdx.x == 0) off[R] = carry;
   __syncthreads();
-  if (s_bad || carry > past_rows) {
+  if (s_bad || (pk != nullptr && carry > past_rows)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, s_bad ? s_bad : FLIDE_ERR_CAPACITY);
     return;
   }
@@ -142,7 +142,7 @@ __global__ void history_gather_kernel(int R, const int32_t *req_slot, int max_re
   const int lane = threadIdx.x & 31;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int i = warp; i < carry; i += nwarps) {
+  for (int i = warp; pk != nullptr && i < carry; i += nwarps) {
     const int r = upper_bound_h(off, R + 1, i) - 1;
     const long pr = pool_row(table, max_blocks, block_rows, req_slot[r], i - off[r]);
     if (pr < 0) {
@@ -245,7 +245,7 @@ int flide_history_append(const flide_tree_index *idx, const int32_t *req_slot,
   using namespace flide;
   if (!idx || !req_slot || !start || !table || !k || !v || !pool_k || !pool_v) return FLIDE_ERR_SHAPE;
   if (max_blocks <= 0 || block_rows <= 0 || Hkv <= 0 || d <= 0) return FLIDE_ERR_SHAPE;
-  const int es = dtype == FLIDE_BF16 ? 2 : dtype == FLIDE_F32 ? 4 : 0;
+  const int es = dtype == FLIDE_BF16 ? 2 : dtype == FLIDE_F32 ? 4 : dtype == FLIDE_E4M3 ? 1 : 0;
   if (!es) return FLIDE_ERR_SHAPE;
   const long row_bytes = (long)Hkv * d * es;
   if (row_bytes % 16) return FLIDE_ERR_SHAPE;
@@ -273,7 +273,8 @@ int flide_history_gather(int32_t R, const int32_t *req_slot, int32_t max_request
   if (max_requests <= 0 || max_blocks <= 0 || block_rows <= 0 || Hkv <= 0 || d <= 0 || past_rows < 0)
     return FLIDE_ERR_SHAPE;
   if (past_rows > 0 && (!past_k || !past_v)) return FLIDE_ERR_SHAPE;
-  const int es = dtype == FLIDE_BF16 ? 2 : dtype == FLIDE_F32 ? 4 : 0;
+  if ((past_k == nullptr) != (past_v == nullptr)) return FLIDE_ERR_SHAPE;
+  const int es = dtype == FLIDE_BF16 ? 2 : dtype == FLIDE_F32 ? 4 : dtype == FLIDE_E4M3 ? 1 : 0;
   if (!es) return FLIDE_ERR_SHAPE;
   const long row_bytes = (long)Hkv * d * es;
   if (row_bytes % 16) return FLIDE_ERR_SHAPE;

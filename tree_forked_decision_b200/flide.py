@@ -33,7 +33,8 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_option_probs", "flide_pool_create", "flide_pool_destroy", "flide_pool_append",
            "flide_pool_release", "flide_pool_length", "flide_pool_free_blocks", "flide_pool_export",
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
-           "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_strerror"]
+           "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_fork_attn_paged",
+           "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -117,6 +118,9 @@ def _lib():
         lib.flide_selftest_wait_timeout.restype = ctypes.c_int
         lib.flide_fork_attn_fp8.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, P, F, P, P]
         lib.flide_fork_attn_fp8.restype = ctypes.c_int
+        lib.flide_fork_attn_paged.argtypes = [P, P, P, P, P, I32, I32, P, I32, P, I32, P, I32, I32,
+                                              I32, I32, P, F, P, P]
+        lib.flide_fork_attn_paged.restype = ctypes.c_int
         lib.flide_amax.argtypes = [P, ctypes.c_int64, I32, P, I32, P]
         lib.flide_amax.restype = ctypes.c_int
         lib.flide_quantize_e4m3.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
@@ -257,6 +261,30 @@ def fork_attn_fp8(q8, k8, v8, index: TreeIndex, scale: float, descale, past_k=No
                                       past_rows, ctypes.byref(index.c), Hq, Hkv, d, _ptr(descale),
                                       float(scale), _ptr(out), _stream(stream)),
            "flide_fork_attn_fp8")
+    return out
+
+
+def fork_attn_paged(q, k, v, index: TreeIndex, scale: float, pool_k, pool_v, block_table,
+                    req_slot, block_rows: int, max_blocks: int, descale=None, out=None,
+                    stream=None):
+    """Fork attention with each request's past rows read in place from a
+    block-paged pool (pool_k/pool_v [n_blocks * block_rows, Hkv, 128], bf16 or
+    e4m3 codes with descale), block_table int32 [n_slots * max_blocks],
+    req_slot int32 [R] on the device.  Returns bf16 [T, Hq, 128]."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    e4m3 = q.dtype in (torch.uint8, torch.float8_e4m3fn)
+    dtype = E4M3 if e4m3 else _dtype_code(q)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+    n_blocks = pool_k.shape[0] // block_rows
+    n_slots = block_table.numel() // max_blocks
+    _check(_lib().flide_fork_attn_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(pool_k), _ptr(pool_v),
+                                        n_blocks, block_rows, _ptr(block_table), max_blocks,
+                                        _ptr(req_slot), n_slots, ctypes.byref(index.c), Hq, Hkv, d,
+                                        dtype, _ptr(descale), float(scale), _ptr(out),
+                                        _stream(stream)),
+           "flide_fork_attn_paged")
     return out
 
 

@@ -18,6 +18,12 @@ block allocator (``flide_pool_*`` in libflide.so).  Per step:
 state_in; ``commit`` reserves blocks for each request's root tokens on the
 host, copies the block table to the device, and appends the root rows and the
 root's end state.  ``release(slot)`` returns a finished request's blocks.
+
+Without the packed copy (block_rows a multiple of 128):
+
+    past_len, state_in = store.resume_lengths(slots)
+    ... flide_tree_build ...
+    o = store.fork_attn_paged(q, k, v, index, scale, slots)   # past read in place
 """
 from __future__ import annotations
 
@@ -98,6 +104,32 @@ class HistoryStore:
             self.dk, self.dv, flide._ptr(past_len), flide._ptr(pk), flide._ptr(pv), past_rows,
             flide._ptr(state_in), flide._ptr(self.status), flide._stream()), "flide_history_gather")
         return past_len, pk, pv, state_in
+
+    def resume_lengths(self, slots):
+        """past_len and GDN state_in for a batch whose request r continues
+        slot slots[r] (-1: no history), without packing the rows: for
+        fork_attn_paged, which reads them in place."""
+        slots = [int(s) for s in slots]
+        R = len(slots)
+        req = torch.tensor(slots, dtype=torch.int32, device=self.device)
+        past_len = torch.zeros(R, dtype=torch.int32, device=self.device)
+        state_in = (torch.empty((R, self.H, self.dv, self.dk), dtype=torch.float32, device=self.device)
+                    if self.H else None)
+        self.status.zero_()
+        flide._check(self._lib.flide_history_gather(
+            R, flide._ptr(req), self.max_requests, flide._ptr(self.lengths), flide._ptr(self.table),
+            self.max_blocks, self.block_rows, flide._ptr(self.pool_k), flide._ptr(self.pool_v),
+            self.Hkv, self.d, flide._dtype_code(self.pool_k), flide._ptr(self.pool_S), self.H,
+            self.dk, self.dv, flide._ptr(past_len), None, None, 0, flide._ptr(state_in),
+            flide._ptr(self.status), flide._stream()), "flide_history_gather")
+        return past_len, state_in
+
+    def fork_attn_paged(self, q, k, v, index: flide.TreeIndex, scale: float, slots, out=None):
+        """Fork attention of a batch whose request r continues slot slots[r],
+        the past rows read in place from this pool's blocks."""
+        req = torch.tensor([int(s) for s in slots], dtype=torch.int32, device=self.device)
+        return flide.fork_attn_paged(q, k, v, index, scale, self.pool_k, self.pool_v, self.table,
+                                     req, self.block_rows, self.max_blocks, out=out)
 
     def commit(self, slots, tree, index: flide.TreeIndex, k, v, node_state=None):
         """Appends request r's root tokens (this step's observation) and its
