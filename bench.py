@@ -374,6 +374,7 @@ def main():
     ap.add_argument("--no-decision", action="store_true", help="skip the decision-scoring timing")
     ap.add_argument("--no-history", action="store_true", help="skip the paged history store timing")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 attention timing")
+    ap.add_argument("--no-bounded", action="store_true", help="skip the memory-bounded GDN timing")
     ap.add_argument("--vocab", type=int, default=8192, help="LM-head vocabulary of the decision leg")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--cpu-pairs", type=int, default=16)
@@ -780,6 +781,49 @@ def main():
                "note": "e4m3 q/k/v with per-tensor scales, P rounded to e4m3, fp32 accumulation; "
                        "peak = 2 x measured bf16 (nominal dense e4m3/bf16 ratio)"}
 
+    # memory-bounded GDN schedule: the same layer with at most a quarter of the
+    # one-shot node-state slots live (roots first, then groups of level-1
+    # subtrees resumed from the roots' states); only where the batch has inner
+    # nodes below its roots
+    bounded = None
+    if not args.no_bounded and g is not None and flide.state_slots(tree) > tree.R:
+        from tree_forked_decision_b200.schedule import BoundedGdn, plan_state_groups
+        full = flide.state_slots(tree)
+        budget = max(-(-full // 4), 1)
+        try:
+            plan_state_groups(tree, budget)
+        except flide.FlideError:
+            budget = full
+        # the schedule of this tree shape is built once, like the step's index
+        bplan = BoundedGdn(tree, budget, g["H"], g["dk"], g["dv"], device=device)
+        n_groups = bplan.groups
+        bo = torch.empty_like(step.go)
+
+        def bnd():
+            bplan.run(step.gq, step.gk, step.gv, step.gg, step.gb, state_in=step.state_in, out=bo)
+
+        for _ in range(max(args.warmup, 1)):
+            bnd()
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            bev[i][0].record()
+            bnd()
+            bev[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        if bplan.status() != 0:
+            raise SystemExit(f"device status {bplan.status()} in the bounded GDN leg")
+        state_b = 4 * g["H"] * g["dk"] * g["dv"]
+        bounded = {"ms": max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in bev), pg, device),
+                   "one_shot_ms": gdn_ms, "slot_budget": budget, "one_shot_slots": full,
+                   "groups": n_groups, "state_bytes": budget * state_b,
+                   "one_shot_state_bytes": full * state_b,
+                   "rel_l2_vs_one_shot": float((bo.float() - step.go.float()).norm() / step.go.float().norm()),
+                   "note": "GDN layer with at most slot_budget node states live: roots, then groups of "
+                           "level-1 subtrees resumed from the roots' states (planned once per tree "
+                           "shape on the host; timed: row gathers, tree builds, GDN launches, scatters)"}
+
     # combined roofline of the step: the layers' roofline times summed, over the
     # measured per-step P50
     combined = None
@@ -820,6 +864,7 @@ def main():
         "decision": decision,
         "history": history,
         "fp8": fp8,
+        "bounded": bounded,
         "gpu_launches": step.launches * args.steps,
         "clocks": clk.summary(),
     }

@@ -435,6 +435,32 @@ int flide_history_gather(int32_t R, const int32_t *req_slot, int32_t max_request
                          int32_t dv, int32_t *past_len, void *past_k, void *past_v,
                          int32_t past_rows, float *state_in, int32_t *status, flide_stream stream);
 
+/* ---- memory-bounded GDN scheduling ---------------------------------------
+ * Memory for cloned states is what limits how many options one call can hold
+ * (techfi24.com, "Limites et perspectives").  Fork = isolation lets each
+ * request's tree be cut below its root: the roots run once and keep their end
+ * states, then whole level-1 subtrees run in groups, each group a batch of its
+ * own whose zero-token roots resume from the kept states (the Python layer's
+ * schedule.fork_gdn_bounded drives these calls).
+ *
+ * Host planner.  req_node_ptr [R+1], parent [N] (request-local, -1 for a
+ * root) are HOST arrays.  Writes node_group[n] = -1 for roots, else the group
+ * of n's level-1 ancestor's subtree; groups hold whole subtrees in stream
+ * order, packed greedily so that each group's batch needs at most max_slots
+ * node-state slots (one per request root in the group, plus its widest odd and
+ * widest even depth's inner nodes, as flide_tree_build assigns them).  Returns
+ * FLIDE_ERR_CAPACITY if one subtree alone needs more, FLIDE_ERR_INVALID for a
+ * malformed tree, FLIDE_ERR_SHAPE for bad arguments. */
+int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
+                            int32_t max_slots, int32_t *node_group, int32_t *n_groups);
+
+/* Device row copy: dst row dst_idx[i] <- src row src_idx[i] for i < n (a NULL
+ * index array means i), rows of row_bytes bytes (a multiple of 4; pointers
+ * 4-byte aligned, 16-byte words when rows and pointers allow).  Index arrays
+ * are device int32.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA. */
+int flide_copy_rows(void *dst, const void *src, const int32_t *dst_idx, const int32_t *src_idx,
+                    int32_t n, int64_t row_bytes, flide_stream stream);
+
 /* Diagnostic, with no counterpart in the pages: runs, in one thread on
  * `stream`, the bounded mbarrier wait that every kernel of this library uses
  * (try_wait with a suspend hint, limit checked against the global timer) on a

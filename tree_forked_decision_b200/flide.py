@@ -34,7 +34,7 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_pool_release", "flide_pool_length", "flide_pool_free_blocks", "flide_pool_export",
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
            "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_fork_attn_paged",
-           "flide_strerror"]
+           "flide_plan_state_groups", "flide_copy_rows", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -121,6 +121,10 @@ def _lib():
         lib.flide_fork_attn_paged.argtypes = [P, P, P, P, P, I32, I32, P, I32, P, I32, P, I32, I32,
                                               I32, I32, P, F, P, P]
         lib.flide_fork_attn_paged.restype = ctypes.c_int
+        lib.flide_plan_state_groups.argtypes = [I32, P, P, I32, P, P]
+        lib.flide_plan_state_groups.restype = ctypes.c_int
+        lib.flide_copy_rows.argtypes = [P, P, P, P, I32, ctypes.c_int64, P]
+        lib.flide_copy_rows.restype = ctypes.c_int
         lib.flide_amax.argtypes = [P, ctypes.c_int64, I32, P, I32, P]
         lib.flide_amax.restype = ctypes.c_int
         lib.flide_quantize_e4m3.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
