@@ -221,46 +221,80 @@ class ClockSampler:
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------
 
-def cpu_oracle_rate(tree, a, g, attn_rows: int, gdn_pairs: int, seed: int = 0):
-    """Times the oracle on a seeded uniform sample of the workload's units --
-    attention query rows and GDN (request, head) pairs -- and scales each time
-    by (all units / sampled units).  Returns (evals/s, description, threads)."""
-    import oracle  # test infrastructure: only this leg and the reference arm use it
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
+
+class OracleSampler:
+    """Times the oracle on seeded uniform samples of the workload's units --
+    attention query rows and GDN (request, head) pairs -- and scales each time
+    by (all units / sampled units).  The inputs are converted to fp32 once."""
+
+    def __init__(self, tree, a, g):
+        import oracle  # test infrastructure: only the CPU-baseline leg and the reference arm use it
+        self.oracle, self.tree, self.a, self.g = oracle, tree, a, g
+        f32 = lambda t: t.float().numpy()
+        if a is not None:
+            self.qa, self.ka, self.va = f32(a["q"]), f32(a["k"]), f32(a["v"])
+            self.pka, self.pva = f32(a["past_k"]), f32(a["past_v"])
+        if g is not None:
+            self.gin = {nm: f32(g[nm]) for nm in ("q", "k", "v", "g", "beta")}
+            self.st = f32(g["state_in"]) if np.any(tree.past_len > 0) else None
+
+    def attention(self, n, rng):
+        """Extrapolated seconds for all query rows, from n sampled rows."""
+        tree, a = self.tree, self.a
+        n_rows = tree.T * a["Hq"]
+        pick = rng.choice(n_rows, size=min(n, n_rows), replace=False)
+        rows = np.stack([pick // a["Hq"], pick % a["Hq"]], 1).astype(np.int32)
+        t0 = time.perf_counter()
+        self.oracle.attention_rows(tree.arrays(), self.qa, self.ka, self.va, self.pka, self.pva,
+                                   1.0 / math.sqrt(a["d"]), rows)
+        return (time.perf_counter() - t0) * n_rows / len(rows), f"{len(rows)} of {n_rows} attention query rows"
+
+    def gdn(self, n, rng):
+        """Extrapolated seconds for all (request, head) pairs, from n sampled pairs."""
+        tree, H = self.tree, self.g["H"]
+        all_pairs = [(r, h) for r in range(tree.R) for h in range(H)]
+        sel = rng.choice(len(all_pairs), size=min(n, len(all_pairs)), replace=False)
+        heads = sorted({all_pairs[i][1] for i in sel})
+        # slice the selected heads so the oracle reads only their data
+        hs = {nm: np.ascontiguousarray(x[:, heads]) for nm, x in self.gin.items()}
+        pairs = [(all_pairs[i][0], heads.index(all_pairs[i][1])) for i in sel]
+        st = np.ascontiguousarray(self.st[:, heads]) if self.st is not None else None
+        t0 = time.perf_counter()
+        self.oracle.gdn(tree.arrays(), hs["q"], hs["k"], hs["v"], hs["g"], hs["beta"], state_in=st,
+                        memoise=True, pairs=pairs)
+        return ((time.perf_counter() - t0) * len(all_pairs) / len(sel),
+                f"{len(sel)} of {len(all_pairs)} GDN (request, head) pairs (memoised oracle)")
+
+    def threads(self):
+        return self.oracle.num_threads()
+
+
+def cpu_oracle_rate(tree, a, g, attn_rows: int, gdn_pairs: int, seed: int = 0):
+    """One sampled timing of the oracle: (evals/s, description, threads)."""
+    smp = OracleSampler(tree, a, g)
     rng = np.random.default_rng(seed)
-    f32 = lambda t: t.float().numpy()
     t_attn = t_gdn = 0.0
     parts = []
     if a is not None:
-        T, Hq = tree.T, a["Hq"]
-        n_rows = T * Hq
-        pick = rng.choice(n_rows, size=min(attn_rows, n_rows), replace=False)
-        rows = np.stack([pick // Hq, pick % Hq], 1).astype(np.int32)
-        qa, ka, va = f32(a["q"]), f32(a["k"]), f32(a["v"])
-        pka, pva = f32(a["past_k"]), f32(a["past_v"])
-        t0 = time.perf_counter()
-        oracle.attention_rows(tree.arrays(), qa, ka, va, pka, pva, 1.0 / math.sqrt(a["d"]), rows)
-        t_attn = (time.perf_counter() - t0) * n_rows / len(rows)
-        del qa, ka, va
-        parts.append(f"{len(rows)} of {n_rows} attention query rows")
+        t_attn, d = smp.attention(attn_rows, rng)
+        parts.append(d)
     if g is not None:
-        H = g["H"]
-        all_pairs = [(r, h) for r in range(tree.R) for h in range(H)]
-        sel = rng.choice(len(all_pairs), size=min(gdn_pairs, len(all_pairs)), replace=False)
-        heads = sorted({all_pairs[i][1] for i in sel})
-        # slice the selected heads so the oracle reads only their data
-        hq = lambda t: np.ascontiguousarray(f32(t)[:, heads])
-        pairs = [(all_pairs[i][0], heads.index(all_pairs[i][1])) for i in sel]
-        st = f32(g["state_in"])[:, heads] if np.any(tree.past_len > 0) else None
-        gq, gk, gv, gg, gb = hq(g["q"]), hq(g["k"]), hq(g["v"]), hq(g["g"]), hq(g["beta"])
-        t0 = time.perf_counter()
-        oracle.gdn(tree.arrays(), gq, gk, gv, gg, gb, state_in=st, memoise=True, pairs=pairs)
-        t_gdn = (time.perf_counter() - t0) * len(all_pairs) / len(sel)
-        parts.append(f"{len(sel)} of {len(all_pairs)} GDN (request, head) pairs (memoised oracle)")
+        t_gdn, d = smp.gdn(gdn_pairs, rng)
+        parts.append(d)
     rate = tree.branch_tokens / (t_attn + t_gdn)
     desc = (" and ".join(parts) + f", seeded uniform sample; each time scaled by all/sampled "
             f"units: attention {t_attn:.1f} s + GDN {t_gdn:.1f} s per step extrapolated")
-    return rate, desc, oracle.num_threads()
+    return rate, desc, smp.threads()
 
 
 # ---------------------------------------------------------------------------
@@ -326,18 +360,42 @@ def job_throughput(units_per_rank: int, steps: int, world: int, ms_max: float) -
 
 
 def run_reference(args):
+    """The oracle as the reference arm: every step times a sample of the
+    workload on the host cores and extrapolates to all of it.  The attention
+    sample shrinks as steps + warm-up grow (the same total over the run); a GDN
+    sample (one (request, head) pair per core, each a whole request's
+    sequence) is taken in about 13 of the steps, evenly spread, and the other
+    steps reuse the latest GDN time, so any --steps/--warmup run ends within a
+    few minutes."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
     tree, a, g, dtype = inputs.make_inputs(args.workload, seed=args.seed)
-    for _ in range(args.warmup):
-        cpu_oracle_rate(tree, a, g, args.ref_rows, args.ref_pairs, seed=1)
-    rates, desc, threads = [], "", 1
-    t_start = time.perf_counter()
-    for s in range(args.steps):
-        r, desc, threads = cpu_oracle_rate(tree, a, g, args.ref_rows, args.ref_pairs, seed=2 + s)
-        rates.append(r)
-    wall = time.perf_counter() - t_start
+    smp = OracleSampler(tree, a, g)
+    total = max(args.steps + args.warmup, 1)
+    rows = max(64, args.ref_rows * 13 // total)
+    pairs = max(args.ref_pairs, smp.threads())
+    t_gdn, gdn_desc, n_gdn = 0.0, "", 0
+    rates, desc = [], ""
+    t_start = None
+    for s_ in range(total):
+        if s_ == args.warmup:
+            t_start = time.perf_counter()
+        rng = np.random.default_rng(2 + s_)
+        t_attn, parts = 0.0, []
+        if a is not None:
+            t_attn, d = smp.attention(rows, rng)
+            parts.append(d)
+        if g is not None and (s_ == 0 or (s_ * 13) // total != ((s_ - 1) * 13) // total):
+            t_gdn, gdn_desc = smp.gdn(pairs, rng)
+            n_gdn += 1
+        if g is not None:
+            parts.append(gdn_desc)
+        if s_ >= args.warmup:
+            rates.append(tree.branch_tokens / (t_attn + t_gdn))
+            desc = (" and ".join(parts) + f" per step (GDN timed in {n_gdn} of {s_ + 1} steps so far, "
+                    f"reused between); each time scaled by all/sampled units")
+    wall = time.perf_counter() - t_start if t_start is not None else 0.0
     value = statistics.median(rates)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
@@ -348,8 +406,8 @@ def run_reference(args):
         "config": {"workload": args.workload, "requests": tree.R, "tokens": tree.T,
                    "branch_tokens": tree.branch_tokens, "seed": args.seed,
                    "oracle": "plain C fp64 oracle (memoised GDN), OpenMP over units"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": smp.threads(), "cpu_model": cpu_model(),
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }
@@ -360,8 +418,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="flide", choices=["flide", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--seed", type=int, default=None)
@@ -874,7 +932,8 @@ def main():
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, desc, threads = cpu_oracle_rate(tree, a, g, args.cpu_rows, args.cpu_pairs)
-        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "cpu_model": cpu_model(), "kind": "oracle",
+               "sample": desc}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
