@@ -52,3 +52,85 @@ def test_graph_bucket_rejects_oversize_tree():
     buckets = GraphBuckets([BucketShape(R=2, N=8, T=100, P=0, D=1)], ATTN, None)
     with pytest.raises(ValueError):
         buckets.pick(inputs.fanout_tree(1, 200, 2, 4))
+
+
+def test_e4m3_and_paged_calls_replay_in_a_graph():
+    """The e4m3 quantisation (amax, codes), the e4m3 attention and the paged
+    attention are asynchronous, allocation-free calls: captured once in a CUDA
+    graph with the tree build, a replay on new input values equals the same
+    calls run eagerly, bit for bit."""
+    tree = inputs.fanout_tree(2, 150, 5, 9, past=200)
+    Hq, Hkv, d, rows_per_block = 8, 2, 128, 128
+    dt = flide.DeviceTree(*tree.arrays(), max_depth=1)
+    idx = flide.TreeIndex(dt.R, dt.N, dt.T, dt.max_depth)
+    scale = 1.0 / math.sqrt(d)
+    dev = lambda t: t.cuda()
+    a = inputs.attn_inputs(tree, Hq, Hkv, d, torch.bfloat16, np.random.default_rng(0))
+    q, k, v, pk, pv = (dev(a[n]) for n in ("q", "k", "v", "past_k", "past_v"))
+    u8 = lambda t: torch.empty(t.shape, dtype=torch.uint8, device="cuda")
+    q8, k8, v8, pk8, pv8 = u8(q), u8(k), u8(v), u8(pk), u8(pv)
+    am = torch.zeros(3, device="cuda")
+    ds = torch.empty(3, device="cuda")
+    o8 = torch.empty_like(q)
+    op = torch.empty_like(q)
+    # pool: request r's past rows in blocks 2r+1, 2r (reversed order), slots 1, 0
+    P = int(tree.past_len[0])
+    nb = -(-P // rows_per_block)
+    pool_k = torch.zeros((2 * tree.R * nb * rows_per_block, Hkv, d), dtype=torch.bfloat16, device="cuda")
+    pool_v = torch.zeros_like(pool_k)
+    table = torch.zeros((tree.R, nb), dtype=torch.int32)
+    slots = torch.tensor(list(range(tree.R))[::-1], dtype=torch.int32)
+    for r in range(tree.R):
+        for b in range(nb):
+            table[slots[r], b] = tree.R * nb + r * nb + (nb - 1 - b)
+    table_d, slots_d = table.view(-1).cuda(), slots.cuda()
+
+    def fill_pool():
+        for r in range(tree.R):
+            for b in range(nb):
+                blk = int(table[slots[r], b])
+                n = min(rows_per_block, P - b * rows_per_block)
+                src = slice(r * P + b * rows_per_block, r * P + b * rows_per_block + n)
+                pool_k[blk * rows_per_block: blk * rows_per_block + n] = pk[src]
+                pool_v[blk * rows_per_block: blk * rows_per_block + n] = pv[src]
+
+    def calls():
+        flide.tree_build(dt, idx)
+        for i, (x, px) in enumerate(((q, None), (k, pk), (v, pv))):
+            flide.amax(x, out=am[i:i + 1])
+            if px is not None:
+                flide.amax(px, out=am[i:i + 1], accumulate=True)
+        for i, (x, x8, px, px8) in enumerate(((q, q8, None, None), (k, k8, pk, pk8), (v, v8, pv, pv8))):
+            flide.quantize_e4m3(x, am[i:i + 1], out=x8, descale=ds[i:i + 1])
+            if px is not None:
+                flide.quantize_e4m3(px, am[i:i + 1], out=px8, descale=None)
+        flide.fork_attn_fp8(q8, k8, v8, idx, scale, ds, past_k=pk8, past_v=pv8, out=o8)
+        flide.fork_attn_paged(q, k, v, idx, scale, pool_k, pool_v, table_d, slots_d, rows_per_block, nb,
+                              out=op)
+
+    fill_pool()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        calls()  # first calls outside the capture (per-device set-up)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        calls()
+    # new values in the same buffers, then replay
+    b = inputs.attn_inputs(tree, Hq, Hkv, d, torch.bfloat16, np.random.default_rng(1))
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (pk, "past_k"), (pv, "past_v")):
+        t.copy_(b[n])
+    fill_pool()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    got = [t.clone() for t in (o8, op, q8, k8, pk8, ds)]
+    calls()
+    torch.cuda.synchronize()
+    assert idx.status() == 0
+    for g_, e_ in zip(got, (o8, op, q8, k8, pk8, ds)):
+        assert torch.equal(g_, e_)
+    # and the replayed paged output equals the packed-past attention on the new values
+    assert torch.equal(got[1], flide.fork_attn(q, k, v, idx, scale, past_k=pk, past_v=pv))
