@@ -68,11 +68,12 @@ def attn_work(tree, a):
     return flops, byts
 
 
-def gdn_work(tree, g):
+def gdn_work(tree, g, esize=None):
     """Algorithmic bytes of one GDN fork scan: q, k, v, out, g, beta once, one
     fp32 state write per saved node (roots and nodes with children), and one
     state read per parent with children (its checkpoint is broadcast to all
-    its branches) and per resumed root."""
+    its branches) and per resumed root.  esize: bytes per q, k, v element when
+    they differ from the output's (e4m3 inputs, bf16 output)."""
     H, dk, dv = g["H"], g["dk"], g["dv"]
     es = 2 if g["q"].dtype == torch.bfloat16 else 4
     state = 4 * H * dk * dv
@@ -85,7 +86,8 @@ def gdn_work(tree, g):
     roots = int(np.sum(rp[1:] > rp[:-1]))
     writes = int(has_child.sum()) + roots - int(sum(has_child[rp[r]] for r in range(tree.R) if rp[r + 1] > rp[r]))
     reads = int(has_child.sum()) + int(np.sum(tree.past_len > 0))
-    return tree.T * H * ((2 * dk + 2 * dv) * es + 8) + state * (writes + reads)
+    io = (2 * dk + 2 * dv) * es if esize is None else (2 * dk + dv) * esize + dv * es
+    return tree.T * H * (io + 8) + state * (writes + reads)
 
 
 # ---------------------------------------------------------------------------
@@ -864,14 +866,57 @@ def main():
         qbytes = elems * (2 + 2 + 1)  # amax read, convert read + write
         peak8 = 2.0 * peak
         diff = (o8.float() - step.o.float()).norm() / step.o.float().norm()
+        gdn8 = {}
+        if g is not None and g["dk"] == 128 and g["dv"] == 128:
+            gam = torch.zeros(3, dtype=torch.float32, device=device)
+            gds = torch.empty(3, dtype=torch.float32, device=device)
+            gq8, gk8, gv8 = u8(step.gq), u8(step.gk), u8(step.gv)
+            go8 = torch.empty_like(step.go)
+            ns8 = torch.empty_like(step.node_state)
+
+            def gquant():
+                for i, (x, x8) in enumerate(((step.gq, gq8), (step.gk, gk8), (step.gv, gv8))):
+                    flide.amax(x, out=gam[i:i + 1])
+                    flide.quantize_e4m3(x, gam[i:i + 1], out=x8, descale=gds[i:i + 1])
+
+            def gdn8_run():
+                flide.fork_gdn_fp8(gq8, gk8, gv8, step.gg, step.gb, step.idx, ns8, gds,
+                                   state_in=step.state_in, out=go8)
+
+            for _ in range(max(args.warmup, 1)):
+                gquant()
+                gdn8_run()
+            gev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+            barrier()
+            for i in range(args.steps):
+                gev[i][0].record()
+                gquant()
+                gev[i][1].record()
+                gdn8_run()
+                gev[i][2].record()
+            torch.cuda.synchronize()
+            barrier()
+            if step.idx.status() != 0:
+                raise SystemExit(f"device status {step.idx.status()} in the fp8 GDN leg")
+            gq_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in gev), pg, device)
+            g8_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in gev), pg, device)
+            gb8 = gdn_work(tree, g, esize=1)
+            gdn8 = {"gdn_ms": g8_ms, "gdn_algorithmic_bytes": gb8, "gdn_gbs": gb8 / (g8_ms / 1000.0) / 1e9,
+                    "gdn_frac_of_hbm_peak": gb8 / (g8_ms / 1000.0) / 1e9 / hbm,
+                    "gdn_speedup_vs_bf16": gdn_ms / g8_ms,
+                    "gdn_quant_ms": gq_ms,
+                    "gdn_rel_l2_vs_bf16_output": float((go8.float() - step.go.float()).norm()
+                                                       / step.go.float().norm())}
         fp8 = {"attn_ms": a8_ms, "tflops": flops / (a8_ms / 1000.0) / 1e12, "peak": peak8,
                "frac_of_tensor_peak": flops / (a8_ms / 1000.0) / 1e12 / peak8,
                "speedup_vs_bf16_attn": (kernels.get("fork_attn") or {}).get("ms", float("nan")) / a8_ms,
                "quant_ms": q_ms, "quant_bytes": qbytes, "quant_gbs": qbytes / (q_ms / 1000.0) / 1e9,
                "quant_frac_of_hbm_peak": qbytes / (q_ms / 1000.0) / 1e9 / hbm,
                "rel_l2_vs_bf16_output": float(diff),
-               "note": "e4m3 q/k/v with per-tensor scales, P rounded to e4m3, fp32 accumulation; "
-                       "peak = 2 x measured bf16 (nominal dense e4m3/bf16 ratio)"}
+               **gdn8,
+               "note": "e4m3 q/k/v with per-tensor scales; attention: P rounded to e4m3, fp32 "
+                       "accumulation, peak = 2 x measured bf16 (nominal dense e4m3/bf16 ratio); GDN: "
+                       "codes converted exactly to bf16 in the kernel, HBM bytes with 1-byte q/k/v"}
 
     # memory-bounded GDN schedule: the same layer with at most a quarter of the
     # one-shot node-state slots live (roots first, then groups of level-1

@@ -223,6 +223,23 @@ int flide_fork_attn_paged(const void *q, const void *k, const void *v, const voi
                           flide_stream stream);
 
 /*
+ * Gated DeltaNet fork scan over e4m3 q, k, v (the pages' FP8 mode; techfi24.com,
+ * "Exact State Forking" and "Performances").  Same recurrence, tree handling,
+ * states and arguments as flide_fork_gdn, with
+ *   q, k [T, H, 128], v [T, H, 128]   e4m3 codes (one byte each)
+ *   descale  device float[3] = {sq, sk, sv}: the values are sq*q, sk*k, sv*v
+ *   out      [T, H, 128] bf16
+ * Tensor-core kernel only (dk = dv = 128), else FLIDE_ERR_SHAPE.  The codes
+ * are converted to bf16 exactly and the descale factors fold into products
+ * the scan forms anyway, so the arithmetic is that of flide_fork_gdn on the
+ * decoded values.  Uses idx->work as scratch.
+ */
+int flide_fork_gdn_fp8(const void *q, const void *k, const void *v, const float *descale,
+                       const float *g, const float *beta, const float *state_in,
+                       flide_tree_index *idx, int32_t H, int32_t dk, int32_t dv, void *out,
+                       float *node_state, int32_t n_state_slots, flide_stream stream);
+
+/*
  * Absolute maximum for per-tensor e4m3 scaling.  *amax (device float) becomes
  * max(|x_i|) over the n elements of x (FLIDE_F32 or FLIDE_BF16, 16-byte
  * aligned), or max(*amax, that) when `accumulate` is non-zero, so several

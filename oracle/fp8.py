@@ -15,6 +15,13 @@ Functions:
   quantize_e4m3(x, amax=None) per-tensor quantisation in the float32 steps
                               inv = 448 / amax, y = x * inv, code = e4m3(y);
                               descale = amax / 448 (amax 0: inv = descale = 1)
+  gdn_fp8(...)                Gated DeltaNet fork scan over decoded fp8 q, k, v
+                              (sq Q, sk K, sv V) with the given gates and
+                              states; the delta rule is not linear in k, so the
+                              decoded values times the descale factors are
+                              formed in float32 (exact for power-of-two
+                              factors, as the tests use) and handed to the
+                              fp64 GDN oracle
   attention_fp8(...)          fork attention over decoded fp8 inputs: with
                               q = sq Q, k = sk K, v = sv V (Q, K, V the decoded
                               codes) the attention of (q, k, v) at softmax
@@ -100,3 +107,13 @@ def attention_fp8(tree, q8, k8, v8, pk8, pv8, descale, scale, rows=None):
     if rows is None:
         return sv * attention_all(tree, Q, K, V, PK, PV, c)
     return sv * attention_rows(tree, Q, K, V, PK, PV, c, rows)
+
+
+def gdn_fp8(tree, q8, k8, v8, g, beta, descale, state_in=None, pairs=None):
+    """Gated DeltaNet fork scan over e4m3 q, k, v with descale factors
+    (sq, sk, sv): float64 [T, H, dv] (zeros outside ``pairs``)."""
+    from . import gdn
+    sq, sk, sv = (np.float32(s) for s in descale)
+    dq = lambda a, s: (decode_e4m3(a).astype(np.float32) * s).astype(np.float32)
+    return gdn(tree, dq(q8, sq), dq(k8, sk), dq(v8, sv), np.asarray(g, np.float32),
+               np.asarray(beta, np.float32), state_in=state_in, pairs=pairs)

@@ -2,7 +2,8 @@
 the format's defining values (OCP 8-bit floating point specification, e4m3),
 PyTorch's own float8_e4m3fn conversion (a library routine) over every code and
 over random in-range values, round-half-to-even ties, saturation, the
-per-tensor scaling steps, and a brute-force fp64 attention on a tiny tree."""
+per-tensor scaling steps, and brute-force fp64 attention and token-by-token
+delta rule on tiny trees."""
 import math
 
 import numpy as np
@@ -134,3 +135,49 @@ def test_attention_fp8_equals_brute_force_on_dequantized_inputs():
     rows = np.array([[0, 0], [T - 1, 3], [6, 1]])
     part = fp8.attention_fp8(tree, q8, k8, v8, pk8, pv8, (sq, sk, sv), scale, rows)
     np.testing.assert_allclose(part, got[rows[:, 0], rows[:, 1]], rtol=0, atol=0)
+
+
+def _brute_gdn(parent, seg, q, k, v, g, beta, s0):
+    """Token-by-token delta rule along each node's isolated path (one request,
+    fp64): S <- alpha (S - beta (S k) k^T) + beta v k^T, o = S q."""
+    starts = np.concatenate([[0], np.cumsum(seg)])
+    T, H, dk = q.shape
+    out = np.zeros((T, H, v.shape[2]))
+    for n in range(len(seg)):
+        chain = []
+        a = n
+        while a >= 0:
+            chain.append(a)
+            a = parent[a]
+        toks = [t for a in reversed(chain) for t in range(starts[a], starts[a + 1])]
+        for h in range(H):
+            S = s0[h].copy()
+            for t in toks:
+                al = np.exp(g[t, h])
+                u = S @ k[t, h]
+                S = al * (S - beta[t, h] * np.outer(u, k[t, h])) + beta[t, h] * np.outer(v[t, h], k[t, h])
+                if starts[n] <= t < starts[n + 1]:
+                    out[t, h] = S @ q[t, h]
+    return out
+
+
+def test_gdn_fp8_equals_brute_force_on_dequantized_inputs():
+    rng = np.random.default_rng(13)
+    parent, seg = [-1, 0, 0, 1], [6, 3, 4, 2]
+    T, H, dk = sum(seg), 2, 8
+    tree = ([0, 4], parent, seg, [1])
+    codes = lambda x, amp: torch.from_numpy((x * amp).astype(np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q8 = codes(unit(rng.standard_normal((T, H, dk))), 256.0)
+    k8 = codes(unit(rng.standard_normal((T, H, dk))), 256.0)
+    v8 = codes(rng.standard_normal((T, H, dk)), 64.0)
+    g = -np.logaddexp(0.0, rng.standard_normal((T, H))).astype(np.float32)
+    beta = (1 / (1 + np.exp(-rng.standard_normal((T, H))))).astype(np.float32)
+    s0 = (rng.standard_normal((1, H, dk, dk)) * 0.1).astype(np.float32)
+    ds = (1 / 256, 1 / 256, 1 / 64)
+    dec = lambda c, s: fp8.decode_e4m3(c) * s
+    want = _brute_gdn(parent, seg, dec(q8, ds[0]), dec(k8, ds[1]), dec(v8, ds[2]),
+                      g.astype(np.float64), beta.astype(np.float64), s0[0].astype(np.float64))
+    got = fp8.gdn_fp8(tree, q8, k8, v8, g, beta, ds, state_in=s0)
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)

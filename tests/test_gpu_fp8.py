@@ -30,7 +30,7 @@ import oracle
 from oracle import fp8 as ofp8
 from tree_forked_decision_b200 import flide, inputs
 
-from gpu_helpers import build
+from gpu_helpers import assert_close, build
 
 pytestmark = pytest.mark.gpu
 
@@ -213,3 +213,80 @@ def test_fullsize_fork_attn_fp8_sampled(name):
     rows = _rows(tree, spec["Hq"], 1500, np.random.default_rng(1))
     want, tol = _oracle_and_bound(tree, a, scale, rows)
     _assert_within(got[rows[:, 0], rows[:, 1]], want, tol)
+
+
+# ---------------------------------------------------------------------------
+# Gated DeltaNet fork scan over e4m3 inputs
+# ---------------------------------------------------------------------------
+
+GDN8_CASES = {
+    "leveled_resume": lambda rng: inputs.leveled_tree(rng, 3, depth_range=(1, 3), options_range=(3, 30),
+                                                      prefix_range=(60, 300), branch_range=(2, 40),
+                                                      n_resume=2),
+    "fanout_long_prefix": lambda rng: inputs.fanout_tree(2, 700, 9, 13, past=5),
+    "deep_chain": lambda rng: inputs._tree([(3, [(-1, 17)] + [(i, 5 + i) for i in range(8)])], 8),
+    "zero_token_root_with_past": lambda rng: inputs._tree([(50, [(-1, 0), (0, 5), (0, 70)]),
+                                                           (0, [(-1, 20), (0, 3)])], 1),
+}
+
+
+def _run_gdn8(tree, g8, H):
+    _, idx = build(tree)
+    dev = {k_: v_.cuda() for k_, v_ in g8.items() if isinstance(v_, torch.Tensor)}
+    has_state = bool(np.any(tree.past_len > 0))
+    node_state = torch.zeros((max(flide.state_slots(tree), 1), H, 128, 128), device="cuda")
+    out = flide.fork_gdn_fp8(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], idx, node_state,
+                             dev["descale"], state_in=dev["state_in"] if has_state else None)
+    torch.cuda.synchronize()
+    assert idx.status() == 0, idx.status()
+    return out, node_state, idx, dev, has_state
+
+
+@pytest.mark.parametrize("case", sorted(GDN8_CASES))
+def test_fork_gdn_fp8_vs_oracle_and_bf16(case):
+    """Against the oracle over the decoded inputs (bf16 bar), and bit for bit
+    against flide_fork_gdn on bf16 inputs holding the same values: e4m3 codes
+    convert exactly, and with power-of-two descale factors folding them into
+    the scan's products changes no rounding."""
+    rng = np.random.default_rng(zlib.crc32(case.encode()) % 1000)
+    tree = GDN8_CASES[case](rng)
+    H = 2
+    g8 = inputs.fp8_gdn_inputs(tree, H, 128, 128, rng, gate_scale=0.1)
+    out, node_state, idx, dev, has_state = _run_gdn8(tree, g8, H)
+    n = lambda t: t.numpy()
+    want = ofp8.gdn_fp8(tree.arrays(), n(g8["q"]), n(g8["k"]), n(g8["v"]), n(g8["g"]), n(g8["beta"]),
+                        n(g8["descale"]), state_in=n(g8["state_in"]) if has_state else None)
+    assert_close(out.float().cpu().numpy(), want, torch.bfloat16)
+    # the bf16 kernel on the decoded values (exact in bf16)
+    ds = g8["descale"].tolist()
+    deq = lambda c, s: (torch.from_numpy(ofp8.decode_e4m3(n(c)) * s).to(torch.bfloat16)).cuda()
+    ns2 = torch.zeros_like(node_state)
+    ref = flide.fork_gdn(deq(g8["q"], ds[0]), deq(g8["k"], ds[1]), deq(g8["v"], ds[2]), dev["g"],
+                         dev["beta"], idx, ns2, state_in=dev["state_in"] if has_state else None)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert torch.equal(node_state, ns2)
+
+
+@pytest.mark.parametrize("name,n_pairs", [("gdn_fanout_bf16", 6), ("large_fanout_bf16", 4)])
+def test_fullsize_fork_gdn_fp8_sampled(name, n_pairs):
+    """The GDN workloads' trees and head counts with e4m3 inputs; every token of
+    sampled (request, head) pairs against the oracle."""
+    tree, _, spec, _, rng = inputs.workload(name)
+    H = spec["H"]
+    g8 = inputs.fp8_gdn_inputs(tree, H, 128, 128, rng, gate_scale=spec["gate_scale"])
+    out, _, _, _, has_state = _run_gdn8(tree, g8, H)
+    got = out.float().cpu().numpy()
+    prng = np.random.default_rng(2)
+    sel = prng.choice(tree.R * H, size=n_pairs, replace=False)
+    heads = sorted({int(i % H) for i in sel})
+    pairs = [(int(i // H), heads.index(int(i % H))) for i in sel]
+    hs = lambda t: np.ascontiguousarray(t.numpy()[:, heads])
+    want = ofp8.gdn_fp8(tree.arrays(), hs(g8["q"]), hs(g8["k"]), hs(g8["v"]), hs(g8["g"]),
+                        hs(g8["beta"]), g8["descale"].numpy(),
+                        state_in=hs(g8["state_in"]) if has_state else None, pairs=pairs)
+    starts = np.concatenate([[0], np.cumsum(tree.seg_len)])
+    rp = tree.req_node_ptr
+    for (r, hi) in pairs:
+        toks = np.arange(starts[rp[r]], starts[rp[r + 1]])
+        assert_close(got[toks, heads[hi]], want[toks, hi], torch.bfloat16)

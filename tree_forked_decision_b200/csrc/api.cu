@@ -20,7 +20,7 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
 bool fork_gdn_tc_supported(int dk, int dv, int dtype);
 int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
                 const float *state_in, const flide_tree_index *x, int H, void *out,
-                float *node_state, int n_slots, cudaStream_t s);
+                float *node_state, int n_slots, cudaStream_t s, int dtype, const float *descale);
 int fork_gdn_portable(const void *q, const void *k, const void *v, const float *g,
                       const float *beta, const float *state_in, const flide_tree_index *x,
                       int H, int dk, int dv, int dtype, void *out, float *node_state,
@@ -173,11 +173,24 @@ int flide_fork_gdn(const void *q, const void *k, const void *v, const float *g,
                    int32_t n_state_slots, int32_t flags, flide_stream stream) {
   if (!idx || !q || !k || !v || !g || !beta || !out || !node_state) return FLIDE_ERR_SHAPE;
   if (H <= 0 || n_state_slots <= 0) return FLIDE_ERR_SHAPE;
+  if (dtype == FLIDE_E4M3) return FLIDE_ERR_SHAPE;  // needs descale factors: flide_fork_gdn_fp8
   if (!(flags & FLIDE_FLAG_PORTABLE) && fork_gdn_tc_supported(dk, dv, dtype))
     return fork_gdn_tc(q, k, v, g, beta, state_in, idx, H, out, node_state, n_state_slots,
-                       (cudaStream_t)stream);
+                       (cudaStream_t)stream, dtype, nullptr);
   return fork_gdn_portable(q, k, v, g, beta, state_in, idx, H, dk, dv, dtype, out, node_state,
                            n_state_slots, (cudaStream_t)stream);
+}
+
+int flide_fork_gdn_fp8(const void *q, const void *k, const void *v, const float *descale,
+                       const float *g, const float *beta, const float *state_in,
+                       flide_tree_index *idx, int32_t H, int32_t dk, int32_t dv, void *out,
+                       float *node_state, int32_t n_state_slots, flide_stream stream) {
+  if (!idx || !q || !k || !v || !descale || !g || !beta || !out || !node_state)
+    return FLIDE_ERR_SHAPE;
+  if (H <= 0 || n_state_slots <= 0) return FLIDE_ERR_SHAPE;
+  if (!fork_gdn_tc_supported(dk, dv, FLIDE_E4M3)) return FLIDE_ERR_SHAPE;
+  return fork_gdn_tc(q, k, v, g, beta, state_in, idx, H, out, node_state, n_state_slots,
+                     (cudaStream_t)stream, FLIDE_E4M3, descale);
 }
 
 int flide_state_save(const flide_tree_index *idx, const void *k, const void *v,

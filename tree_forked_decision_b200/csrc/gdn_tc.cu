@@ -36,6 +36,9 @@
 // first, from a shared counter.  Every wait is bounded (2 s).
 #include <cstddef>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -75,6 +78,7 @@ enum { B_FULL = 0, B_MMA = 2, NUM_BARS = 3 };
 
 struct GdnTcParams {
   flide_tree_index x;
+  const float *descale;  // e4m3 inputs: {q, k, v} descale factors
   const float *g, *beta, *state_in;
   __nv_bfloat16 *out;
   float *node_state;
@@ -210,6 +214,35 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
   return v;
 }
 
+// e4m3 inputs (F8): a chunk's K, Q and V arrive as e4m3 codes (64 rows of 128
+// bytes each) in one staging buffer that aliases the fp32 A / T area, and are
+// converted to bf16 (exactly: every e4m3 value is a bf16 value) into the same
+// swizzled tiles the bf16 path loads; the next chunk's codes are loaded after
+// the current chunk's solve has finished with A and T.  The descale factors
+// fold into products the kernel forms anyway: A and (M o QK^T) take sk^2 and
+// sq sk, T' (for W) sk, T'' (for U) sv, Delta' (state update) sk, and the
+// output's Q S0^T term sq -- so no extra rounding is added.
+constexpr int SM_STAGE8 = SM_A;  // e4m3 staging: K rows at +0, Q at +8192, V at +16384
+static_assert(SM_STAGE8 % 1024 == 0 && SM_STAGE8 + 3 * 8192 <= SM_X,
+              "e4m3 staging must be 1024-aligned and end before the block-product area");
+
+// 16 e4m3 codes (one 16-byte chunk) to 16 floats, exactly
+__device__ __forceinline__ void decode16_e4m3(uint4 raw, float (&f)[16]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const __half2_raw hr =
+          __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> (16 * h2)), __NV_E4M3);
+      const float2 f2 = __half22float2(__half2(hr));
+      f[4 * i + 2 * h2] = f2.x;
+      f[4 * i + 2 * h2 + 1] = f2.y;
+    }
+  }
+}
+
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const GdnTcParams p) {
@@ -220,6 +253,8 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int lg = warp & 3, wg = warp >> 2;  // TMEM lane group; column half
   const int row = lg * 32 + lane;           // this thread's TMEM lane = tile row
   const flide_tree_index &x = p.x;
+  const float dsq = F8 ? p.descale[0] : 1.f, dsk = F8 ? p.descale[1] : 1.f,
+              dsv = F8 ? p.descale[2] : 1.f;
   float *sbeta = reinterpret_cast<float *>(smem + SM_SCAL);
   float *sG = sbeta + C;
   float *sgam = sG + C;
@@ -337,6 +372,15 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // K, Q, V of chunk c into stage st (thread 0)
     auto issue_loads = [&](int c, int st) {
       const int row = tbeg + c * C;
+      if (F8) {  // codes into the one staging buffer
+        const uint32_t sg = sb + SM_STAGE8, fb = bar(B_FULL + 0);
+        pending0 = true;
+        mbar_arrive_expect_tx(fb, 3 * 8192);
+        tma_load_3d(sg, &tm_k, fb, 0, h, row);
+        tma_load_3d(sg + 8192, &tm_q, fb, 0, h, row);
+        tma_load_3d(sg + 16384, &tm_v, fb, 0, h, row);
+        return;
+      }
       const uint32_t kq = sb + SM_KQ + st * 32768, vv = sb + SM_V + st * 16384;
       const uint32_t fb = bar(B_FULL + st);
       if (st == 0) pending0 = true; else pending1 = true;
@@ -369,8 +413,9 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int n = min(C, tend - cbeg);
       const bool update = scan && (c + 1 < nchunks || slot >= 0);
       const uint32_t kq = sb + SM_KQ + st * 32768, vv = sb + SM_V + st * 16384;
-      // prefetch the next chunk into the other stage (its last readers are done)
-      if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1, st ^ 1);
+      // prefetch the next chunk into the other stage (its last readers are
+      // done); e4m3 codes wait until this chunk's solve has freed the staging
+      if (!F8 && tid == 0 && c + 1 < nchunks) issue_loads(c + 1, st ^ 1);
       __syncwarp();
 
       // ---- per-token scalars: beta, segment id, then the segmented log decay
@@ -411,13 +456,33 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         sG2[2 * lane + 1] = g1 * 1.4426950408889634f;
       }
       // ---- wait for this chunk's K, Q, V
-      const bool loaded = mbar_wait(bar(B_FULL + st), st == 0 ? full_phase0 : full_phase1, vabort,
+      const int fbi = F8 ? 0 : st;
+      const bool loaded = mbar_wait(bar(B_FULL + fbi), fbi == 0 ? full_phase0 : full_phase1, vabort,
                                     kTimeoutNs);
       if (loaded) {
-        if (st == 0) { full_phase0 ^= 1; pending0 = false; }
+        if (fbi == 0) { full_phase0 ^= 1; pending0 = false; }
         else { full_phase1 ^= 1; pending1 = false; }
       }
       if (!__syncthreads_and(loaded)) { ok = false; break; }
+      if (F8) {
+        // e4m3 codes -> bf16 tiles of stage st: staging row rr (K 0-63, Q
+        // 64-127, V 128-191), 16-code chunk j = dims 16j .. 16j+15
+        const uint8_t *stg = smem + SM_STAGE8;
+        for (int e = tid; e < 3 * C * 8; e += kThreads) {
+          const int rr = e >> 3, j = e & 7;
+          const uint4 raw = *reinterpret_cast<const uint4 *>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
+          float f[16];
+          decode16_e4m3(raw, f);
+          const int which = rr >> 6, t = rr & (C - 1), slab = j >> 2, cc = (j & 3) * 2;
+          uint8_t *dst = which < 2 ? smem + SM_KQ + st * 32768 + slab * 16384
+                                   : smem + SM_V + st * 16384 + slab * 8192;
+          const int R = which == 1 ? t + C : t;
+          st_chunk(dst, R, cc, pack8(f));
+          st_chunk(dst, R, cc + 1, pack8(f + 8));
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+      }
       const float gam_last = sgam[n - 1];
 
       // ---- R1 = [K;Q] [K;Q]^T
@@ -460,7 +525,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_ld32(tl + R1 + 32 * wg, d1);
         const int i = row & (C - 1);
         const bool is_a = row < C;
-        const float G2i = sG2[i], scale_i = is_a ? sbeta[i] : 1.f;
+        const float G2i = sG2[i], scale_i = is_a ? sbeta[i] * (dsk * dsk) : dsq * dsk;
         const int si = sseg[i];
         const int jmax = is_a ? i - 1 : i;  // last visible j
         const float4 *g4 = reinterpret_cast<const float4 *>(sG2);
@@ -565,8 +630,8 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int u = 0; u < 8; ++u) {
               const int j = 16 * qq + 8 * q + u;
               const float tv = (j >> 4) <= (i >> 4) ? Tm[i * A_LD + j] : 0.f;
-              f1[u] = tv * sbeta[j] * sgam[j];
-              f2[u] = tv * sbeta[j];
+              f1[u] = F8 ? tv * (sbeta[j] * sgam[j] * dsk) : tv * sbeta[j] * sgam[j];
+              f2[u] = F8 ? tv * (sbeta[j] * dsv) : tv * sbeta[j];
             }
             st_chunk(t1, i, 2 * qq + q, pack8(f1));
             st_chunk(t2, i, 2 * qq + q, pack8(f2));
@@ -575,6 +640,8 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       fence_proxy_async_smem();
       __syncthreads();
+      // the staging area (A, T) is free now: the next chunk's e4m3 codes
+      if (F8 && tid == 0 && c + 1 < nchunks) issue_loads(c + 1, 0);
 
       // ---- R2 = T' K (= W),  R3 = T'' V (= U)
       if (tid == 0) {
@@ -628,7 +695,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_ld64(tl + R3 + wg * 64, dr);
         uint8_t *db = smem + SM_S0 + wg * 8192;
         __nv_bfloat16 *dat = reinterpret_cast<__nv_bfloat16 *>(smem + SM_S0 + 16384);
-        const float sc = gam_last / sgam[j];
+        const float sc = F8 ? gam_last / sgam[j] * dsk : gam_last / sgam[j];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           float f[8];
@@ -665,7 +732,7 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int i = row - C;
         const bool valid = i < n && cbeg + i < Tact;
         __nv_bfloat16 *o = p.out + ((size_t)(cbeg + i) * p.H + h) * D;
-        const float gi = sgam[i];
+        const float gi = F8 ? sgam[i] * dsq : sgam[i];
         {
           const int half = wg;  // this warp's 64 output dims
           uint32_t o1[32], o2[32];
@@ -744,15 +811,17 @@ EncodeTiledFn encode_fn_gdn() {
   return fn;
 }
 
-// [rows, heads, 128] bf16 as a 3-D tensor (dim, head, row); box 64 x 1 x 64
-bool make_map_gdn(CUtensorMap *m, const void *base, int heads, long rows) {
+// [rows, heads, 128] bf16 (esz 2) or e4m3 (esz 1) as a 3-D tensor (dim, head,
+// row); box of 128 bytes of dims x 1 x 64 rows
+bool make_map_gdn(CUtensorMap *m, const void *base, int heads, long rows, int esz) {
   EncodeTiledFn enc = encode_fn_gdn();
   if (!enc || rows <= 0) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {256, (cuuint64_t)heads * 256};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)C};
+  cuuint64_t strides[2] = {(cuuint64_t)128 * esz, (cuuint64_t)heads * 128 * esz};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / esz), 1, (cuuint32_t)C};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+  return enc(m, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(base), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -760,29 +829,36 @@ bool make_map_gdn(CUtensorMap *m, const void *base, int heads, long rows) {
 }  // namespace
 
 bool fork_gdn_tc_supported(int dk, int dv, int dtype) {
-  return dtype == FLIDE_BF16 && dk == D && dv == D && encode_fn_gdn() != nullptr;
+  return (dtype == FLIDE_BF16 || dtype == FLIDE_E4M3) && dk == D && dv == D &&
+         encode_fn_gdn() != nullptr;
 }
 
 int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, const float *beta,
                 const float *state_in, const flide_tree_index *x, int H, void *out,
-                float *node_state, int n_slots, cudaStream_t s) {
+                float *node_state, int n_slots, cudaStream_t s, int dtype, const float *descale) {
+  const bool f8 = dtype == FLIDE_E4M3;
+  if (f8 && !descale) return FLIDE_ERR_SHAPE;
+  const int esz = f8 ? 1 : 2;
   CUtensorMap mq, mk, mv;
   const long T = x->T > 0 ? x->T : 1;
-  if (!make_map_gdn(&mq, q, H, T) || !make_map_gdn(&mk, k, H, T) || !make_map_gdn(&mv, v, H, T))
+  if (!make_map_gdn(&mq, q, H, T, esz) || !make_map_gdn(&mk, k, H, T, esz) ||
+      !make_map_gdn(&mv, v, H, T, esz))
     return FLIDE_ERR_CUDA;
-  static bool attr_set[64] = {};
+  static bool attr_set[2][64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLIDE_ERR_CUDA;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    if (cudaFuncSetAttribute(gdn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return FLIDE_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  if (dev < 0 || dev >= 64 || !attr_set[f8][dev]) {
+    const cudaError_t e =
+        f8 ? cudaFuncSetAttribute(gdn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
+           : cudaFuncSetAttribute(gdn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return FLIDE_ERR_CUDA;
+    if (dev >= 0 && dev < 64) attr_set[f8][dev] = true;
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   GdnTcParams prm;
   prm.x = *x;
+  prm.descale = descale;
   prm.g = g;
   prm.beta = beta;
   prm.state_in = state_in;
@@ -795,7 +871,10 @@ int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, con
     prm.level = lvl;
     gdn_groups_kernel<<<1, 1024, 0, s>>>(*x, lvl, prm.goff);
     FLIDE_LAUNCH_CHECK();
-    gdn_tc_kernel<<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
+    if (f8)
+      gdn_tc_kernel<true><<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
+    else
+      gdn_tc_kernel<false><<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
     FLIDE_LAUNCH_CHECK();
   }
   return FLIDE_OK;

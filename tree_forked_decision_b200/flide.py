@@ -34,7 +34,7 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_pool_release", "flide_pool_length", "flide_pool_free_blocks", "flide_pool_export",
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
            "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_fork_attn_paged",
-           "flide_plan_state_groups", "flide_copy_rows", "flide_strerror"]
+           "flide_plan_state_groups", "flide_copy_rows", "flide_fork_gdn_fp8", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -125,6 +125,8 @@ def _lib():
         lib.flide_plan_state_groups.restype = ctypes.c_int
         lib.flide_copy_rows.argtypes = [P, P, P, P, I32, ctypes.c_int64, P]
         lib.flide_copy_rows.restype = ctypes.c_int
+        lib.flide_fork_gdn_fp8.argtypes = [P, P, P, P, P, P, P, P, I32, I32, I32, P, P, I32, P]
+        lib.flide_fork_gdn_fp8.restype = ctypes.c_int
         lib.flide_amax.argtypes = [P, ctypes.c_int64, I32, P, I32, P]
         lib.flide_amax.restype = ctypes.c_int
         lib.flide_quantize_e4m3.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
@@ -289,6 +291,27 @@ def fork_attn_paged(q, k, v, index: TreeIndex, scale: float, pool_k, pool_v, blo
                                         dtype, _ptr(descale), float(scale), _ptr(out),
                                         _stream(stream)),
            "flide_fork_attn_paged")
+    return out
+
+
+def fork_gdn_fp8(q8, k8, v8, g, beta, index: TreeIndex, node_state, descale, state_in=None,
+                 out=None, stream=None):
+    """GDN fork scan over e4m3 codes (uint8 tensors q, k [T, H, 128], v
+    [T, H, 128]); descale is a float32 device tensor [3] = (sq, sk, sv).
+    Returns bf16 [T, H, 128]."""
+    T, H, dk = q8.shape
+    dv = v8.shape[2]
+    for t in (q8, k8, v8):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_contiguous():
+            raise TypeError("e4m3 inputs must be contiguous uint8 / float8_e4m3fn tensors")
+    if descale.dtype != torch.float32 or descale.numel() < 3:
+        raise TypeError("descale must be a float32 tensor of 3 entries")
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=torch.bfloat16, device=q8.device)
+    _check(_lib().flide_fork_gdn_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(descale), _ptr(g),
+                                     _ptr(beta), _ptr(state_in), ctypes.byref(index.c), H, dk, dv,
+                                     _ptr(out), _ptr(node_state), node_state.shape[0],
+                                     _stream(stream)), "flide_fork_gdn_fp8")
     return out
 
 

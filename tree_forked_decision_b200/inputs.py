@@ -263,6 +263,25 @@ def gdn_inputs(tree: Tree, H: int, dk: int, dv: int, dtype: torch.dtype,
                 state_in=torch.from_numpy(state))
 
 
+def fp8_gdn_inputs(tree: Tree, H: int, dk: int, dv: int, rng: np.random.Generator,
+                   gate_scale: float = 1.0, state_scale: float = 0.1,
+                   amp_qk: float = 256.0, amp_v: float = 64.0):
+    """The values of gdn_inputs (float32) with q, k and v as e4m3 codes (uint8
+    tensors) of amp * value, cast by torch's float8_e4m3fn conversion, and
+    descale = (1/amp_qk, 1/amp_qk, 1/amp_v) (float32 [3]); L2-normalised q, k
+    times 256 and N(0,1) v times 64 stay below the format's largest value 448.
+    g, beta and state_in as in gdn_inputs."""
+    d = gdn_inputs(tree, H, dk, dv, torch.float32, rng, gate_scale=gate_scale,
+                   state_scale=state_scale)
+
+    def codes(x, amp):
+        return (x * np.float32(amp)).to(torch.float8_e4m3fn).view(torch.uint8)
+
+    d.update(q=codes(d["q"], amp_qk), k=codes(d["k"], amp_qk), v=codes(d["v"], amp_v),
+             descale=torch.tensor([1.0 / amp_qk, 1.0 / amp_qk, 1.0 / amp_v], dtype=torch.float32))
+    return d
+
+
 # ---------------------------------------------------------------------------
 # Named workloads.  Each returns (tree, attention spec or None, GDN spec or
 # None, dtype).  seed defaults to the workload's index.
