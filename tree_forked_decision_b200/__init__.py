@@ -32,13 +32,14 @@ flattened token stream; parent ids are request-local, -1 for the root):
     torch.cuda.synchronize(); assert idx.status() == 0   # device-detected errors
 
 (``dt_host_tree`` above is any object whose ``arrays()`` returns the four host
-arrays, e.g. ``inputs.Tree``.)  Further calls: ``fork_attn_fp8`` with
-``amax`` / ``quantize_e4m3`` (e4m3 inputs), ``fork_attn_paged`` and
+arrays, e.g. ``inputs.Tree``.)  Further calls: ``fork_attn_fp8`` and
+``fork_gdn_fp8`` with ``amax`` / ``quantize_e4m3`` (e4m3 inputs), ``fork_attn_paged`` and
 ``history.HistoryStore`` (growing histories in a block pool),
 ``branch_logprob`` / ``option_probs`` (decision probabilities over the
 options), ``schedule.BoundedGdn`` (GDN under a node-state memory budget) and
 ``graphs.GraphBuckets`` (captured CUDA graphs per shape bucket).
 """
 from .flide import (DeviceTree, FlideError, TreeIndex, amax, branch_logprob,  # noqa: F401
-                    fork_attn, fork_attn_fp8, fork_attn_paged, fork_gdn, load, option_probs,
+                    fork_attn, fork_attn_fp8, fork_attn_paged, fork_gdn, fork_gdn_fp8, load,
+                    option_probs,
                     quantize_e4m3, state_resume, state_save, state_slots, tree_build)
