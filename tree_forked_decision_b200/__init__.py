@@ -25,14 +25,13 @@ flattened token stream; parent ids are request-local, -1 for the root):
 
     # Gated DeltaNet layer: q, k, v [T,H,128] bf16, g = log(alpha), beta [T,H] fp32;
     # node_state holds the roots' and inner nodes' end states
-    node_state = torch.empty(flide.state_slots(dt_host_tree), 16, 128, 128, device="cuda")
+    node_state = torch.empty(flide.state_slots(dt), 16, 128, 128, device="cuda")
     go = flide.fork_gdn(gq, gk, gv, g, beta, idx, node_state)
 
     flide.state_save(...)   # the prefix becomes checkpointed history for the next step
     torch.cuda.synchronize(); assert idx.status() == 0   # device-detected errors
 
-(``dt_host_tree`` above is any object whose ``arrays()`` returns the four host
-arrays, e.g. ``inputs.Tree``.)  Further calls: ``fork_attn_fp8`` and
+Further calls: ``fork_attn_fp8`` and
 ``fork_gdn_fp8`` with ``amax`` / ``quantize_e4m3`` (e4m3 inputs), ``fork_attn_paged`` and
 ``history.HistoryStore`` (growing histories in a block pool),
 ``branch_logprob`` / ``option_probs`` (decision probabilities over the

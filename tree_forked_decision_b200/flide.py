@@ -197,6 +197,7 @@ class DeviceTree:
     def __init__(self, req_node_ptr, parent, seg_len, past_len, max_depth: int,
                  N: int | None = None, T: int | None = None, device="cuda"):
         as_i32 = lambda a: torch.as_tensor(np.asarray(a, np.int32)).to(device)
+        self._host = tuple(np.asarray(a, np.int32) for a in (req_node_ptr, parent, seg_len, past_len))
         self.req_node_ptr = as_i32(req_node_ptr)
         self.parent = as_i32(parent)
         self.seg_len = as_i32(seg_len)
@@ -214,10 +215,18 @@ class DeviceTree:
                      max_depth: int) -> "DeviceTree":
         """Wraps preallocated int32 device buffers (capacities N, T) without copying."""
         t = cls.__new__(cls)
+        t._host = None
         t.req_node_ptr, t.parent, t.seg_len, t.past_len = req_node_ptr, parent, seg_len, past_len
         t.R = req_node_ptr.shape[0] - 1
         t.N, t.T, t.max_depth = int(N), int(T), int(max_depth)
         return t
+
+    def arrays(self):
+        """The host arrays (req_node_ptr, parent, seg_len, past_len) the tree was
+        built from (for host-side sizing such as state_slots)."""
+        if self._host is None:
+            raise ValueError("a DeviceTree wrapping device buffers has no host arrays")
+        return self._host
 
     def desc(self) -> TreeDesc:
         return TreeDesc(self.R, self.N, self.T, self.max_depth, self.req_node_ptr.data_ptr(),
