@@ -823,54 +823,64 @@ def main():
     # attention, against the e4m3 tensor peak = 2 x the measured bf16 one (the
     # nominal dense ratio of the two formats).
     fp8 = None
-    if not args.no_fp8 and a is not None and a["q"].dtype == torch.bfloat16 and a["d"] == 128:
-        am = torch.zeros(3, dtype=torch.float32, device=device)
-        ds = torch.empty(3, dtype=torch.float32, device=device)
-        u8 = lambda t: None if t is None else torch.empty(t.shape, dtype=torch.uint8, device=device)
-        q8, k8, v8, pk8, pv8 = u8(step.q), u8(step.k), u8(step.v), u8(step.pk), u8(step.pv)
-        o8 = torch.empty_like(step.q)
+    attn_ok = a is not None and a["q"].dtype == torch.bfloat16 and a["d"] == 128
+    gdn_ok = g is not None and g["q"].dtype == torch.bfloat16 and g["dk"] == 128 and g["dv"] == 128
+    if not args.no_fp8 and (attn_ok or gdn_ok):
+        att8, gdn8 = {}, {}
+        u8g = lambda t: torch.empty(t.shape, dtype=torch.uint8, device=device)
+        if attn_ok:
+            am = torch.zeros(3, dtype=torch.float32, device=device)
+            ds = torch.empty(3, dtype=torch.float32, device=device)
+            u8 = lambda t: None if t is None else torch.empty(t.shape, dtype=torch.uint8, device=device)
+            q8, k8, v8, pk8, pv8 = u8(step.q), u8(step.k), u8(step.v), u8(step.pk), u8(step.pv)
+            o8 = torch.empty_like(step.q)
 
-        def quant():
-            for i, (x, px) in enumerate(((step.q, None), (step.k, step.pk), (step.v, step.pv))):
-                flide.amax(x, out=am[i:i + 1])
-                if px is not None:
-                    flide.amax(px, out=am[i:i + 1], accumulate=True)
-            for i, (x, x8, px, px8) in enumerate(((step.q, q8, None, None), (step.k, k8, step.pk, pk8),
-                                                  (step.v, v8, step.pv, pv8))):
-                flide.quantize_e4m3(x, am[i:i + 1], out=x8, descale=ds[i:i + 1])
-                if px is not None:
-                    flide.quantize_e4m3(px, am[i:i + 1], out=px8, descale=None)
+            def quant():
+                for i, (x, px) in enumerate(((step.q, None), (step.k, step.pk), (step.v, step.pv))):
+                    flide.amax(x, out=am[i:i + 1])
+                    if px is not None:
+                        flide.amax(px, out=am[i:i + 1], accumulate=True)
+                for i, (x, x8, px, px8) in enumerate(((step.q, q8, None, None), (step.k, k8, step.pk, pk8),
+                                                      (step.v, v8, step.pv, pv8))):
+                    flide.quantize_e4m3(x, am[i:i + 1], out=x8, descale=ds[i:i + 1])
+                    if px is not None:
+                        flide.quantize_e4m3(px, am[i:i + 1], out=px8, descale=None)
 
-        def attn8():
-            flide.fork_attn_fp8(q8, k8, v8, step.idx, step.scale, ds, past_k=pk8, past_v=pv8, out=o8)
+            def attn8():
+                flide.fork_attn_fp8(q8, k8, v8, step.idx, step.scale, ds, past_k=pk8, past_v=pv8, out=o8)
 
-        for _ in range(max(args.warmup, 1)):
-            quant()
-            attn8()
-        qev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        barrier()
-        for i in range(args.steps):
-            qev[i][0].record()
-            quant()
-            qev[i][1].record()
-            attn8()
-            qev[i][2].record()
-        torch.cuda.synchronize()
-        barrier()
-        if step.idx.status() != 0:
-            raise SystemExit(f"device status {step.idx.status()} in the fp8 leg")
-        q_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in qev), pg, device)
-        a8_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in qev), pg, device)
-        flops = attn_work(tree, a)[0]
-        elems = sum(t.numel() for t in (step.q, step.k, step.v, step.pk, step.pv) if t is not None)
-        qbytes = elems * (2 + 2 + 1)  # amax read, convert read + write
-        peak8 = 2.0 * peak
-        diff = (o8.float() - step.o.float()).norm() / step.o.float().norm()
-        gdn8 = {}
-        if g is not None and g["dk"] == 128 and g["dv"] == 128:
+            for _ in range(max(args.warmup, 1)):
+                quant()
+                attn8()
+            qev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+            barrier()
+            for i in range(args.steps):
+                qev[i][0].record()
+                quant()
+                qev[i][1].record()
+                attn8()
+                qev[i][2].record()
+            torch.cuda.synchronize()
+            barrier()
+            if step.idx.status() != 0:
+                raise SystemExit(f"device status {step.idx.status()} in the fp8 leg")
+            q_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in qev), pg, device)
+            a8_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in qev), pg, device)
+            flops = attn_work(tree, a)[0]
+            elems = sum(t.numel() for t in (step.q, step.k, step.v, step.pk, step.pv) if t is not None)
+            qbytes = elems * (2 + 2 + 1)  # amax read, convert read + write
+            peak8 = 2.0 * peak
+            diff = (o8.float() - step.o.float()).norm() / step.o.float().norm()
+            att8 = {"attn_ms": a8_ms, "tflops": flops / (a8_ms / 1000.0) / 1e12, "peak": peak8,
+                    "frac_of_tensor_peak": flops / (a8_ms / 1000.0) / 1e12 / peak8,
+                    "speedup_vs_bf16_attn": (kernels.get("fork_attn") or {}).get("ms", float("nan")) / a8_ms,
+                    "quant_ms": q_ms, "quant_bytes": qbytes, "quant_gbs": qbytes / (q_ms / 1000.0) / 1e9,
+                    "quant_frac_of_hbm_peak": qbytes / (q_ms / 1000.0) / 1e9 / hbm,
+                    "rel_l2_vs_bf16_output": float(diff)}
+        if gdn_ok:
             gam = torch.zeros(3, dtype=torch.float32, device=device)
             gds = torch.empty(3, dtype=torch.float32, device=device)
-            gq8, gk8, gv8 = u8(step.gq), u8(step.gk), u8(step.gv)
+            gq8, gk8, gv8 = u8g(step.gq), u8g(step.gk), u8g(step.gv)
             go8 = torch.empty_like(step.go)
             ns8 = torch.empty_like(step.node_state)
 
@@ -907,13 +917,7 @@ def main():
                     "gdn_quant_ms": gq_ms,
                     "gdn_rel_l2_vs_bf16_output": float((go8.float() - step.go.float()).norm()
                                                        / step.go.float().norm())}
-        fp8 = {"attn_ms": a8_ms, "tflops": flops / (a8_ms / 1000.0) / 1e12, "peak": peak8,
-               "frac_of_tensor_peak": flops / (a8_ms / 1000.0) / 1e12 / peak8,
-               "speedup_vs_bf16_attn": (kernels.get("fork_attn") or {}).get("ms", float("nan")) / a8_ms,
-               "quant_ms": q_ms, "quant_bytes": qbytes, "quant_gbs": qbytes / (q_ms / 1000.0) / 1e9,
-               "quant_frac_of_hbm_peak": qbytes / (q_ms / 1000.0) / 1e9 / hbm,
-               "rel_l2_vs_bf16_output": float(diff),
-               **gdn8,
+        fp8 = {**att8, **gdn8,
                "note": "e4m3 q/k/v with per-tensor scales; attention: P rounded to e4m3, fp32 "
                        "accumulation, peak = 2 x measured bf16 (nominal dense e4m3/bf16 ratio); GDN: "
                        "codes converted exactly to bf16 in the kernel, HBM bytes with 1-byte q/k/v"}
