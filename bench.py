@@ -782,7 +782,10 @@ def main():
         # attention reading the past in place from the blocks, against the same
         # attention over the packed copy
         tree_w, keep = inputs.warm_variant(tree)
-        if tree_w.P_past == rows and a["d"] == 128 and step.q.dtype == torch.bfloat16:
+        run_paged = float(tree_w.P_past == rows and a["d"] == 128 and step.q.dtype == torch.bfloat16)
+        if pg is not None:  # the same legs on every rank (they hold barriers)
+            run_paged = -max_over_ranks(-run_paged, pg, device)
+        if run_paged > 0:
             ridx = torch.from_numpy(keep).to(device)
             qw, kw, vw = (t[ridx].contiguous() for t in (step.q, step.k, step.v))
             dtw = flide.DeviceTree(*tree_w.arrays(), max_depth=max(tree_w.levels, 1), device=device)
@@ -927,7 +930,12 @@ def main():
     # subtrees resumed from the roots' states); only where the batch has inner
     # nodes below its roots
     bounded = None
-    if not args.no_bounded and g is not None and flide.state_slots(tree) > tree.R:
+    # every rank takes the same legs (each has barriers): the leg runs only if
+    # every rank's batch has inner nodes below its roots
+    run_bounded = float(not args.no_bounded and g is not None and flide.state_slots(tree) > tree.R)
+    if pg is not None:
+        run_bounded = -max_over_ranks(-run_bounded, pg, device)
+    if run_bounded > 0:
         from tree_forked_decision_b200.schedule import BoundedGdn, plan_state_groups
         full = flide.state_slots(tree)
         budget = max(-(-full // 4), 1)
