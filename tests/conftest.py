@@ -11,6 +11,15 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: large-size case (minutes)")
+    # a fresh checkout has no libflide.so: build it (nvcc cross-compiles for
+    # sm_100a without a GPU) so the ABI and host-logic tests can load it
+    from tree_forked_decision_b200 import build as flide_build
+    if not os.path.exists(flide_build.LIB):
+        try:
+            flide_build._nvcc()
+        except RuntimeError:
+            return  # no toolchain: the tests that need the library report it
+        flide_build.build()
 
 
 def pytest_collection_modifyitems(config, items):
