@@ -205,6 +205,54 @@ __device__ __forceinline__ uint32_t sw_elem(int row, int col) {
   return row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2;
 }
 
+// 16 x 16 x 16 block products of the triangular solve on the warp's tensor
+// path: mma.sync m16n8k8 with tf32 inputs (rounded to nearest) and fp32
+// accumulation.  Fragments (g = lane / 4, t = lane % 4): A rows g, g+8 and
+// columns t, t+4 of each 8-wide K step; B rows t, t+4 of the step and column
+// g of each 8-wide N tile; the accumulator holds rows g, g+8 and columns 2t,
+// 2t+1 of each N tile.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// acc += A (16 x 16, row stride lda) B (16 x 16, row stride ldb), fp32 in shared memory
+__device__ __forceinline__ void block_mma16(float (&acc)[2][4], const float *A, int lda, const float *B,
+                                            int ldb, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kk = 0; kk < 16; kk += 8) {
+    const uint32_t a0 = to_tf32(A[g * lda + kk + t]), a1 = to_tf32(A[(g + 8) * lda + kk + t]);
+    const uint32_t a2 = to_tf32(A[g * lda + kk + t + 4]), a3 = to_tf32(A[(g + 8) * lda + kk + t + 4]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const uint32_t b0 = to_tf32(B[(kk + t) * ldb + 8 * nt + g]);
+      const uint32_t b1 = to_tf32(B[(kk + t + 4) * ldb + 8 * nt + g]);
+      mma_tf32_16x8x8(acc[nt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+}
+// stores s * acc (accumulator layout) as a 16 x 16 block with row stride ld
+__device__ __forceinline__ void block_store16(float *C, int ld, const float (&acc)[2][4], float s,
+                                              int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    C[g * ld + 8 * nt + 2 * t] = s * acc[nt][0];
+    C[g * ld + 8 * nt + 2 * t + 1] = s * acc[nt][1];
+    C[(g + 8) * ld + 8 * nt + 2 * t] = s * acc[nt][2];
+    C[(g + 8) * ld + 8 * nt + 2 * t + 1] = s * acc[nt][3];
+  }
+}
+
 __device__ __forceinline__ uint4 pack8(const float *f) {
   uint4 v;
   v.x = pack_bf16x2(f[0], f[1]);
@@ -579,44 +627,24 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           for (int i = 0; i < 16; ++i) Tm[(r0 + i) * A_LD + r0 + cc] = tcol[i];
         }
         __syncthreads();
-        // block row bi: X_bj = sum_{k=j}^{bi-1} A_bk T_kj, then T_bj = -T_bb X_bj.
-        // Thread -> (row r of the block row, column cc) for every column block
-        // j < bi: up to three independent sums.
-        {
-          const int r = tid >> 4, cc = tid & 15;
-          for (int bi = 1; bi < 4; ++bi) {
-            const float *arow = Am + (16 * bi + r) * A_LD;
-            float acc[3] = {0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kb = 0; kb < 3; ++kb) {
-              if (kb >= bi) break;
-#pragma unroll
-              for (int m = 0; m < 16; ++m) {
-                const float a = arow[16 * kb + m];
-                const float *trow = Tm + (16 * kb + m) * A_LD + cc;
-#pragma unroll
-                for (int jb = 0; jb < 3; ++jb)
-                  if (jb <= kb) acc[jb] = fmaf(a, trow[16 * jb], acc[jb]);
-              }
-            }
-#pragma unroll
-            for (int jb = 0; jb < 3; ++jb)
-              if (jb < bi) Xm[(jb * 16 + r) * X_LD + cc] = acc[jb];
-            __syncthreads();
-            const float *trow = Tm + (16 * bi + r) * A_LD + 16 * bi;
-            acc[0] = acc[1] = acc[2] = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-              const float tv = m <= r ? trow[m] : 0.f;
-#pragma unroll
-              for (int jb = 0; jb < 3; ++jb)
-                if (jb < bi) acc[jb] = fmaf(tv, Xm[(jb * 16 + m) * X_LD + cc], acc[jb]);
-            }
-#pragma unroll
-            for (int jb = 0; jb < 3; ++jb)
-              if (jb < bi) Tm[(16 * bi + r) * A_LD + 16 * jb + cc] = -acc[jb];
-            __syncthreads();
+        // block row bi: X_bj = sum_{k=j}^{bi-1} A_bk T_kj, then T_bj = -T_bb X_bj
+        // (T_bb is exactly zero above its diagonal), one warp per column block
+        // j < bi, the 16 x 16 products on the warp's tensor path; X goes
+        // through the warp's scratch block to change fragment layout
+        for (int bi = 1; bi < 4; ++bi) {
+          if (warp < bi) {
+            const int j = warp;
+            float acc[2][4] = {};
+            for (int k = j; k < bi; ++k)
+              block_mma16(acc, Am + 16 * bi * A_LD + 16 * k, A_LD, Tm + 16 * k * A_LD + 16 * j, A_LD, lane);
+            float *xs = Xm + j * 16 * X_LD;
+            block_store16(xs, X_LD, acc, 1.f, lane);
+            __syncwarp();
+            float acc2[2][4] = {};
+            block_mma16(acc2, Tm + 16 * bi * A_LD + 16 * bi, A_LD, xs, X_LD, lane);
+            block_store16(Tm + 16 * bi * A_LD + 16 * j, A_LD, acc2, -1.f, lane);
           }
+          __syncthreads();
         }
         // T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles:
         // thread -> (row i, half of the columns)
