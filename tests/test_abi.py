@@ -5,7 +5,6 @@ import os
 import re
 import subprocess
 
-import pytest
 
 from tree_forked_decision_b200 import flide
 

@@ -10,7 +10,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 from oracle import fp8
 
 

@@ -5,12 +5,11 @@ row of query head 0, plus random rows), GDN on every token of sampled
 (request, head) pairs."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from tree_forked_decision_b200 import inputs
 
-from gpu_helpers import assert_close, build, run_attn, run_gdn
+from gpu_helpers import assert_close, run_attn, run_gdn
 
 pytestmark = pytest.mark.gpu
 

@@ -2,7 +2,6 @@
 same seeded inputs.  Indices bit-exact; fp32 outputs within 1e-4 max-abs;
 bf16 outputs within 2e-2 max-abs and 1e-2 relative L2."""
 import json
-import math
 import os
 import zlib
 
@@ -13,7 +12,7 @@ import torch
 import oracle
 from tree_forked_decision_b200 import flide, inputs
 
-from gpu_helpers import (assert_close, build, device_tree, oracle_attn, oracle_gdn, run_attn,
+from gpu_helpers import (assert_close, build, oracle_attn, oracle_gdn, run_attn,
                          run_gdn)
 
 pytestmark = pytest.mark.gpu
