@@ -474,6 +474,27 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       if (c + 1 < nchunks) load_scalars(c + 1);
       __syncthreads();
+      // bf16 copy of S0 (B operand, rows = dv), made by warps 1-7 while warp 0
+      // scans the gates; warp 4 (same TMEM lanes as warp 0) also takes warp
+      // 0's half.  The state is final: the last chunk's products completed.
+      auto copy_s0_half = [&](int half) {
+        uint32_t sr[64];
+        tc_fence_after();  // warp 4 reads the half warp 0 wrote at the item's start
+        tmem_ld64(tl + R_S + half * 64, sr);
+        uint8_t *s0 = smem + SM_S0 + half * 16384;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
+          st_chunk(s0, row, q, pack8(f));
+        }
+      };
+      if (warp != 0) {
+        copy_s0_half(wg);
+        if (warp == 4) copy_s0_half(0);
+        tc_fence_before();  // warp 0 rescales its half after the next barrier
+      }
       if (warp == 0) {
         // segmented inclusive scan of g, two tokens per lane: (value,
         // segment-start flag) pairs combined Hillis-Steele style
@@ -545,23 +566,14 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
       __syncwarp();
-      // ---- meanwhile: bf16 copy of S0 (B operand, rows = dv); rescale S
-      {
+      // ---- meanwhile: S scaled by gamma_last in TMEM (the bf16 copy of S0
+      //      above was taken from the unscaled state)
+      if (update) {
         uint32_t sr[64];
         tmem_ld64(tl + R_S + wg * 64, sr);
-        uint8_t *s0 = smem + SM_S0 + wg * 16384;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float f[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
-          st_chunk(s0, row, q, pack8(f));
-        }
-        if (update) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) sr[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
-          tmem_st64(tl + R_S + wg * 64, sr);
-        }
+        for (int i = 0; i < 64; ++i) sr[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
+        tmem_st64(tl + R_S + wg * 64, sr);
       }
       if (!mma_sync()) { ok = false; break; }
 
@@ -631,25 +643,12 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // (T_bb is exactly zero above its diagonal), one warp per column block
         // j < bi, the 16 x 16 products on the warp's tensor path; X goes
         // through the warp's scratch block to change fragment layout
-        for (int bi = 1; bi < 4; ++bi) {
-          if (warp < bi) {
-            const int j = warp;
-            float acc[2][4] = {};
-            for (int k = j; k < bi; ++k)
-              block_mma16(acc, Am + 16 * bi * A_LD + 16 * k, A_LD, Tm + 16 * k * A_LD + 16 * j, A_LD, lane);
-            float *xs = Xm + j * 16 * X_LD;
-            block_store16(xs, X_LD, acc, 1.f, lane);
-            __syncwarp();
-            float acc2[2][4] = {};
-            block_mma16(acc2, Tm + 16 * bi * A_LD + 16 * bi, A_LD, xs, X_LD, lane);
-            block_store16(Tm + 16 * bi * A_LD + 16 * j, A_LD, acc2, -1.f, lane);
-          }
-          __syncthreads();
-        }
-        // T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles:
-        // thread -> (row i, half of the columns)
-        {
-          const int i = tid >> 2, qq = tid & 3;  // row, quarter of the columns
+        // T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles, one
+        // 16-row block row at a time (64 items: row, quarter of the columns):
+        // block row b - 1 is converted by two otherwise idle warps while
+        // block row b is solved
+        auto convert_block_row = [&](int b, int item) {
+          const int i = 16 * b + (item >> 2), qq = item & 3;
           uint8_t *t1 = smem + SM_TA, *t2 = smem + SM_TA + 16384;
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
@@ -664,7 +663,24 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             st_chunk(t1, i, 2 * qq + q, pack8(f1));
             st_chunk(t2, i, 2 * qq + q, pack8(f2));
           }
+        };
+        for (int bi = 1; bi < 4; ++bi) {
+          if (warp >= 3 && warp < 5) convert_block_row(bi - 1, tid - 96);
+          if (warp < bi) {
+            const int j = warp;
+            float acc[2][4] = {};
+            for (int k = j; k < bi; ++k)
+              block_mma16(acc, Am + 16 * bi * A_LD + 16 * k, A_LD, Tm + 16 * k * A_LD + 16 * j, A_LD, lane);
+            float *xs = Xm + j * 16 * X_LD;
+            block_store16(xs, X_LD, acc, 1.f, lane);
+            __syncwarp();
+            float acc2[2][4] = {};
+            block_mma16(acc2, Tm + 16 * bi * A_LD + 16 * bi, A_LD, xs, X_LD, lane);
+            block_store16(Tm + 16 * bi * A_LD + 16 * j, A_LD, acc2, -1.f, lane);
+          }
+          __syncthreads();
         }
+        if (tid < 64) convert_block_row(3, tid);
       }
       fence_proxy_async_smem();
       __syncthreads();
