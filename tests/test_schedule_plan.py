@@ -4,7 +4,8 @@ its level-1 ancestor, groups follow stream order, each group's batch (per
 request a zero-token root plus the group's subtrees) needs at most the budget
 of node-state slots by the slot rule flide_tree_build applies, packing is
 greedy (the next group's first subtree would not have fitted), and a subtree
-that alone exceeds the budget, or a malformed tree, is refused."""
+that alone exceeds the budget, or a malformed tree, is refused; the Python
+side's batches cover every token row once."""
 import numpy as np
 import pytest
 
@@ -96,3 +97,37 @@ def test_refuses_malformed_trees_and_bad_budgets():
     assert lib.flide_plan_state_groups(1, p(rp), p(good), 0, p(out), ctypes.byref(ng)) == flide.ERR_SHAPE
     assert lib.flide_plan_state_groups(1, p(rp), p(good), 1, p(out), ctypes.byref(ng)) == flide.OK
     assert ng.value == 1 and out.tolist() == [-1, 0, 0]
+
+
+@pytest.mark.parametrize("case", sorted(TREES))
+def test_batches_cover_every_token_row_once(case):
+    """schedule._batches (host): root batches hold every request's root rows,
+    group batches every other node's rows, each row exactly once; a group's
+    batch rebuilds the subtrees with request-local parents (zero-token roots),
+    and every batch fits the budget by the index builder's slot rule."""
+    from tree_forked_decision_b200.schedule import _batches
+    rng = np.random.default_rng(11)
+    tree = TREES[case](rng)
+    rp, _parent, seg, _ = tree.arrays()
+    for budget in (3, 7, 50):
+        try:
+            batches = _batches(tree, budget)
+        except flide.FlideError:
+            continue
+        seen = np.zeros(tree.T, int)
+        for kind, batch, req_ids in batches:
+            assert flide.state_slots(batch) <= budget
+            brp, bpar, bseg, _ = batch.arrays()
+            assert len(req_ids) == len(brp) - 1 and int(bseg.sum()) == len(batch.rows)
+            seen[batch.rows] += 1
+            if kind == "roots":
+                assert all(p == -1 for p in bpar) and len(bpar) == len(req_ids)
+                assert list(bseg) == [int(seg[rp[r]]) for r in req_ids]
+            else:
+                for bi, r in enumerate(req_ids):
+                    nodes = range(brp[bi], brp[bi + 1])
+                    assert bpar[brp[bi]] == -1 and bseg[brp[bi]] == 0   # zero-token root
+                    for n in nodes:
+                        if n > brp[bi]:
+                            assert 0 <= bpar[n] < n - brp[bi]            # parent precedes
+        assert (seen == 1).all()
