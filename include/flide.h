@@ -161,7 +161,8 @@ int flide_tree_build(const flide_tree_desc *desc, flide_tree_index *idx,
  * dtype FLIDE_F32 or FLIDE_BF16.  With bf16, d == 128, 128 % (Hq/Hkv) == 0 and
  * idx->max_depth <= 8 the tensor-core kernel runs (tcgen05 MMA, TMA, TMEM);
  * otherwise, or with FLIDE_FLAG_PORTABLE, the portable kernel (d a multiple of
- * 32, <= 256).
+ * 32, <= 256).  FLIDE_E4M3 inputs need descale factors and go through
+ * flide_fork_attn_fp8 (FLIDE_ERR_SHAPE here).
  * Uses idx->work as scratch.  Host errors: FLIDE_ERR_SHAPE, FLIDE_ERR_CUDA.
  */
 int flide_fork_attn(const void *q, const void *k, const void *v,
@@ -308,7 +309,9 @@ int flide_fork_attn_noalloc(const void *q, const void *k, const void *v,
  *   out [T, H, dv] dtype
  *   node_state [n_state_slots, H, dv, dk] fp32 (required)
  * Device error FLIDE_ERR_CAPACITY if the tree needs more than n_state_slots.
- * Supported: dk in {32, 64, 128, 256}, dv a multiple of 32.
+ * Supported: dk in {32, 64, 128, 256}, dv a multiple of 32; bf16 with
+ * dk = dv = 128 runs on the tensor cores.  FLIDE_E4M3 inputs go through
+ * flide_fork_gdn_fp8 (FLIDE_ERR_SHAPE here).
  */
 int flide_fork_gdn(const void *q, const void *k, const void *v,
                    const float *g, const float *beta, const float *state_in,
