@@ -474,27 +474,6 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       if (c + 1 < nchunks) load_scalars(c + 1);
       __syncthreads();
-      // bf16 copy of S0 (B operand, rows = dv), made by warps 1-7 while warp 0
-      // scans the gates; warp 4 (same TMEM lanes as warp 0) also takes warp
-      // 0's half.  The state is final: the last chunk's products completed.
-      auto copy_s0_half = [&](int half) {
-        uint32_t sr[64];
-        tc_fence_after();  // warp 4 reads the half warp 0 wrote at the item's start
-        tmem_ld64(tl + R_S + half * 64, sr);
-        uint8_t *s0 = smem + SM_S0 + half * 16384;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float f[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
-          st_chunk(s0, row, q, pack8(f));
-        }
-      };
-      if (warp != 0) {
-        copy_s0_half(wg);
-        if (warp == 4) copy_s0_half(0);
-        tc_fence_before();  // warp 0 rescales its half after the next barrier
-      }
       if (warp == 0) {
         // segmented inclusive scan of g, two tokens per lane: (value,
         // segment-start flag) pairs combined Hillis-Steele style
@@ -566,14 +545,23 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
       __syncwarp();
-      // ---- meanwhile: S scaled by gamma_last in TMEM (the bf16 copy of S0
-      //      above was taken from the unscaled state)
-      if (update) {
+      // ---- meanwhile: bf16 copy of S0 (B operand, rows = dv); rescale S
+      {
         uint32_t sr[64];
         tmem_ld64(tl + R_S + wg * 64, sr);
+        uint8_t *s0 = smem + SM_S0 + wg * 16384;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) sr[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
-        tmem_st64(tl + R_S + wg * 64, sr);
+        for (int q = 0; q < 8; ++q) {
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
+          st_chunk(s0, row, q, pack8(f));
+        }
+        if (update) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) sr[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
+          tmem_st64(tl + R_S + wg * 64, sr);
+        }
       }
       if (!mma_sync()) { ok = false; break; }
 
