@@ -180,3 +180,17 @@ def test_gdn_fp8_equals_brute_force_on_dequantized_inputs():
                       g.astype(np.float64), beta.astype(np.float64), s0[0].astype(np.float64))
     got = fp8.gdn_fp8(tree, q8, k8, v8, g, beta, ds, state_in=s0)
     np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-12)
+
+
+def test_fp8_input_generators_emit_no_nan_codes():
+    """The seeded e4m3 generators clamp before casting, so no code is NaN even
+    for values beyond the format's range; shapes follow the tree."""
+    from tree_forked_decision_b200 import inputs
+    tree = inputs.fanout_tree(2, 40, 3, 5, past=7)
+    a = inputs.fp8_attn_inputs(tree, 4, 2, 16, np.random.default_rng(0), amp=400.0)
+    g = inputs.fp8_gdn_inputs(tree, 2, 16, 16, np.random.default_rng(1), amp_v=400.0)
+    for t in (a["q"], a["k"], a["v"], a["past_k"], a["past_v"], g["q"], g["k"], g["v"]):
+        c = t.numpy()
+        assert c.dtype == np.uint8 and not np.any((c & 0x7F) == 0x7F)
+    assert a["q"].shape == (tree.T, 4, 16) and a["past_k"].shape == (tree.P_past, 2, 16)
+    assert np.isclose(a["descale"].numpy(), 1 / 400.0).all()

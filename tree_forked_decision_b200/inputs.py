@@ -220,12 +220,13 @@ def fp8_attn_inputs(tree: Tree, Hq: int, Hkv: int, d: int, rng: np.random.Genera
     """e4m3 codes (uint8 tensors) of amp * N(0,1) for q [T,Hq,d], k, v [T,Hkv,d]
     and past_k, past_v [sum(past),Hkv,d], cast by torch's float8_e4m3fn
     conversion, with descale = (1/amp, 1/amp, 1/amp) (float32 [3]): the
-    decoded values are N(0,1) to within the format's rounding.  amp * 6 stays
-    below the format's largest value 448 for these sample sizes."""
+    decoded values are N(0,1) to within the format's rounding.  Values are
+    clamped to +-448 first (the cast would make NaN of anything larger; at
+    amp = 64 that takes a 7-sigma draw)."""
     T, P = tree.T, tree.P_past
 
     def codes(shape):
-        x = normals(rng, shape) * np.float32(amp)
+        x = np.clip(normals(rng, shape) * np.float32(amp), -448.0, 448.0)
         return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8)
 
     return dict(q=codes((T, Hq, d)), k=codes((T, Hkv, d)), v=codes((T, Hkv, d)),
@@ -274,8 +275,8 @@ def fp8_gdn_inputs(tree: Tree, H: int, dk: int, dv: int, rng: np.random.Generato
     d = gdn_inputs(tree, H, dk, dv, torch.float32, rng, gate_scale=gate_scale,
                    state_scale=state_scale)
 
-    def codes(x, amp):
-        return (x * np.float32(amp)).to(torch.float8_e4m3fn).view(torch.uint8)
+    def codes(x, amp):  # clamped to +-448: the cast makes NaN of larger values
+        return (x * np.float32(amp)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
 
     d.update(q=codes(d["q"], amp_qk), k=codes(d["k"], amp_qk), v=codes(d["v"], amp_v),
              descale=torch.tensor([1.0 / amp_qk, 1.0 / amp_qk, 1.0 / amp_v], dtype=torch.float32))
