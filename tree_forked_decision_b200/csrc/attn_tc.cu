@@ -747,6 +747,7 @@ extern "C" int flide_fork_attn_noalloc(const void *q, const void *k, const void 
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || past_rows < 0) return FLIDE_ERR_SHAPE;
   if ((past_k == nullptr) != (past_v == nullptr)) return FLIDE_ERR_SHAPE;
   if (past_k == nullptr) past_rows = 0;
+  if (dtype == FLIDE_E4M3) return FLIDE_ERR_SHAPE;  // needs descale factors: flide_fork_attn_fp8
   if (idx->R < 0 || idx->R > kNoAllocMaxRequests) return FLIDE_ERR_CAPACITY;
   if (!(flags & FLIDE_FLAG_PORTABLE) && fork_attn_tc_supported(idx, Hq, Hkv, d, dtype)) {
     int32_t *work = noalloc_work_ptr();

@@ -151,17 +151,20 @@ int state_save(const flide_tree_index *x, const void *k, const void *v, const vo
   if (!x) return FLIDE_ERR_SHAPE;
   const int es = dtype == FLIDE_BF16 ? 2 : (dtype == FLIDE_F32 ? 4 : 0);
   if (!es) return FLIDE_ERR_SHAPE;
+  // every argument is checked before the first launch, so a refused call
+  // leaves the checkpoint untouched
+  const long row_bytes = (long)Hkv * d * es;
+  if (Hkv > 0 && (d <= 0 || row_bytes % 16 != 0 || row_bytes > (1 << 30) || !k || !v || !ck || !cv))
+    return FLIDE_ERR_SHAPE;
+  if (H > 0 && (!node_state || !cS || dk <= 0 || dv <= 0 || ((long)dk * dv) % 4 != 0))
+    return FLIDE_ERR_SHAPE;
   if (Hkv > 0) {
-    const long row_bytes = (long)Hkv * d * es;
-    if (d <= 0 || row_bytes % 16 != 0 || row_bytes > (1 << 30) || !k || !v || !ck || !cv)
-      return FLIDE_ERR_SHAPE;
     save_kv_kernel<<<148 * 4, 256, 0, s>>>(*x, (const char *)k, (const char *)v,
                                            (const char *)pk, (const char *)pv, (int)row_bytes,
                                            (char *)ck, (char *)cv, ckpt_rows);
     FLIDE_LAUNCH_CHECK();
   }
   if (H > 0) {
-    if (!node_state || !cS || ((long)dk * dv) % 4 != 0) return FLIDE_ERR_SHAPE;
     save_state_kernel<<<148 * 4, 256, 0, s>>>(*x, node_state, H, dk * dv, cS);
     FLIDE_LAUNCH_CHECK();
   }
