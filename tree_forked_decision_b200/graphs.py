@@ -44,24 +44,30 @@ class GraphBucket:
         self.shape = s = shape
         self.attn_spec, self.gdn_spec = attn, gdn
         self.device = device
+        self._alloc(dtype)
+        self.dt = flide.DeviceTree.from_buffers(self.req_node_ptr, self.parent, self.seg_len,
+                                                self.past_len, s.N, s.T, s.D)
+        self.idx = flide.TreeIndex(s.R, s.N, s.T, s.D, device=device)
+        self.graph = None
+
+    def _alloc(self, dtype):
+        """The static buffers, sized by the bucket's capacities."""
+        s, device = self.shape, self.device
         i32 = lambda n: torch.zeros(max(n, 1), dtype=torch.int32, device=device)
         self.req_node_ptr = i32(s.R + 1)
         self.parent = i32(s.N)
         self.seg_len = i32(s.N)
         self.past_len = i32(s.R)
-        self.dt = flide.DeviceTree.from_buffers(self.req_node_ptr, self.parent, self.seg_len,
-                                                self.past_len, s.N, s.T, s.D)
-        self.idx = flide.TreeIndex(s.R, s.N, s.T, s.D, device=device)
         z = lambda *shp, dt=dtype: torch.zeros(shp, dtype=dt, device=device)
-        if attn:
-            Hq, Hkv, d = attn["Hq"], attn["Hkv"], attn["d"]
+        if self.attn_spec:
+            Hq, Hkv, d = self.attn_spec["Hq"], self.attn_spec["Hkv"], self.attn_spec["d"]
             self.q, self.k, self.v = z(s.T, Hq, d), z(s.T, Hkv, d), z(s.T, Hkv, d)
             self.past_k, self.past_v = z(max(s.P, 1), Hkv, d), z(max(s.P, 1), Hkv, d)
             self.out = z(s.T, Hq, d)
             self.ckpt_k, self.ckpt_v = z(s.P + s.T, Hkv, d), z(s.P + s.T, Hkv, d)
             self.scale = 1.0 / math.sqrt(d)
-        if gdn:
-            H, dk, dv = gdn["H"], gdn["dk"], gdn["dv"]
+        if self.gdn_spec:
+            H, dk, dv = self.gdn_spec["H"], self.gdn_spec["dk"], self.gdn_spec["dv"]
             self.gq, self.gk, self.gv = z(s.T, H, dk), z(s.T, H, dk), z(s.T, H, dv)
             self.gg = z(s.T, H, dt=torch.float32)
             self.gb = z(s.T, H, dt=torch.float32)
@@ -69,7 +75,6 @@ class GraphBucket:
             self.gout = z(s.T, H, dv)
             self.node_state = z(s.N, H, dv, dk, dt=torch.float32)
             self.ckpt_S = z(s.R, H, dv, dk, dt=torch.float32)
-        self.graph = None
 
     def _sequence(self):
         flide.tree_build(self.dt, self.idx)
