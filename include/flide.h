@@ -414,6 +414,16 @@ void flide_pool_destroy(flide_pool *pool);
  * before the call); -FLIDE_ERR_CAPACITY when blocks run out or the request's
  * table is full, -FLIDE_ERR_INVALID for a bad slot.  Nothing changes on error. */
 int64_t flide_pool_append(flide_pool *pool, int32_t slot, int32_t n);
+/* One step's appends, all or nothing: for i < n, request slots[i] gains
+ * counts[i] rows (slots[i] = -1: skipped, starts[i] = -1) and starts[i]
+ * receives the history row where they start.  A request listed more than once
+ * gets its appends in list order.  The whole batch is checked first, so on
+ * error no request changes: FLIDE_ERR_CAPACITY when the blocks or a request's
+ * table would run out (or a length would pass INT32_MAX), FLIDE_ERR_INVALID
+ * for a slot >= max_requests or a negative count, FLIDE_ERR_SHAPE for NULL
+ * arrays with n > 0.  Host arrays. */
+int flide_pool_append_batch(flide_pool *pool, int32_t n, const int32_t *slots,
+                            const int32_t *counts, int32_t *starts);
 /* Returns all blocks of request `slot` to the free list; its length becomes 0. */
 int flide_pool_release(flide_pool *pool, int32_t slot);
 /* History rows held by `slot` (negative status for a bad slot). */
@@ -428,7 +438,8 @@ int flide_pool_export(const flide_pool *pool, int32_t *table, int32_t *lengths);
  * [start[r], start[r] + root length) of its slot through the block table, and
  * its root's end state node_state[state_slot[root]] to pool_S[req_slot[r]]
  * (when node_state and pool_S are given).  start[r] is what flide_pool_append
- * returned.  A row without a block sets FLIDE_ERR_CAPACITY in idx->status.
+ * returned (or flide_pool_append_batch wrote).  A row without a block sets
+ * FLIDE_ERR_CAPACITY in idx->status.
  * All arrays are device memory; row bytes (Hkv d element size) % 16 == 0. */
 int flide_history_append(const flide_tree_index *idx, const int32_t *req_slot,
                          const int32_t *start, const int32_t *table, int32_t max_blocks,

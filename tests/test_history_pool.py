@@ -1,6 +1,7 @@
 """The native block allocator behind the multi-step history store (host only,
 no GPU): reservations, block reuse after release, capacity errors that leave
-the state unchanged, and invariants under a random sequence of operations."""
+the state unchanged, invariants under a random sequence of operations, and
+the all-or-nothing batch append that a step's commit uses."""
 import ctypes
 
 import numpy as np
@@ -88,3 +89,105 @@ def test_random_operations_keep_invariants(lib):
                 assert (table[r, :nb] >= 0).all() and (table[r, nb:] == -1).all()
     finally:
         lib.flide_pool_destroy(pool)
+
+
+def _batch(lib, pool, slots, counts):
+    sl, ct = np.array(slots, np.int32), np.array(counts, np.int32)
+    starts = np.full(len(slots), -7, np.int32)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    return lib.flide_pool_append_batch(pool, len(slots), p(sl), p(ct), p(starts)), starts
+
+
+def test_batch_append_all_or_nothing(lib):
+    pool = lib.flide_pool_create(6, 4, 4, 4)
+    try:
+        st, starts = _batch(lib, pool, [0, 1, -1, 0], [5, 3, 9, 2])
+        assert st == flide.OK and starts.tolist() == [0, 0, -1, 5]   # slot 0 twice, in order
+        before = _export(lib, pool, 4, 4)
+        assert before[1].tolist() == [7, 3, 0, 0] and lib.flide_pool_free_blocks(pool) == 3
+        for slots, counts, code in [
+            ([2, 3], [8, 8], flide.ERR_CAPACITY),        # 4 blocks wanted, 3 free
+            ([1, 1], [10, 5], flide.ERR_CAPACITY),       # 18 rows = 5 blocks > a table's 4
+            ([2, 4], [1, 1], flide.ERR_INVALID),         # slot >= max_requests
+            ([2, 3], [1, -1], flide.ERR_INVALID),        # negative count
+        ]:
+            st, starts = _batch(lib, pool, slots, counts)
+            assert st == code
+            assert (starts == -7).all()                  # nothing written on error
+            after = _export(lib, pool, 4, 4)
+            assert np.array_equal(after[0], before[0]) and np.array_equal(after[1], before[1])
+            assert lib.flide_pool_free_blocks(pool) == 3
+        assert lib.flide_pool_append_batch(pool, 2, None, None, None) == flide.ERR_SHAPE
+        assert lib.flide_pool_append_batch(pool, 0, None, None, None) == flide.OK
+        st, starts = _batch(lib, pool, [2, 3, 2], [4, 4, 4])          # exactly the 3 free blocks
+        assert st == flide.OK and starts.tolist() == [0, 0, 4] and lib.flide_pool_free_blocks(pool) == 0
+    finally:
+        lib.flide_pool_destroy(pool)
+
+
+def test_random_batches_match_sequential_appends(lib):
+    """A batch that succeeds equals its appends made one by one; a batch that
+    fails is exactly one whose one-by-one appends would fail somewhere, and it
+    leaves the pool as it was."""
+    rng = np.random.default_rng(1)
+    n_blocks, rows, R, mb = 30, 8, 5, 10
+    pool = lib.flide_pool_create(n_blocks, rows, R, mb)
+    length, nblk = np.zeros(R, int), np.zeros(R, int)
+    try:
+        for _ in range(300):
+            if rng.random() < 0.15:
+                s = int(rng.integers(0, R))
+                assert lib.flide_pool_release(pool, s) == flide.OK
+                length[s], nblk[s] = 0, 0
+                continue
+            k = int(rng.integers(0, 5))
+            slots = rng.integers(-1, R, k).tolist()
+            counts = rng.integers(0, 30, k).tolist()
+            # the model: the appends one by one
+            ln, nb, free, ok, want = length.copy(), nblk.copy(), n_blocks - int(nblk.sum()), True, []
+            for s, c in zip(slots, counts):
+                if s < 0:
+                    want.append(-1)
+                    continue
+                need = -(-(ln[s] + c) // rows)
+                if need > mb or need - nb[s] > free:
+                    ok = False
+                    break
+                want.append(int(ln[s]))
+                free -= need - nb[s]
+                ln[s], nb[s] = ln[s] + c, need
+            before = _export(lib, pool, R, mb)
+            st, starts = _batch(lib, pool, slots, counts)
+            if ok:
+                assert st == flide.OK and starts.tolist() == want
+                length, nblk = ln, nb
+            else:
+                assert st == flide.ERR_CAPACITY
+                after = _export(lib, pool, R, mb)
+                assert np.array_equal(after[0], before[0]) and np.array_equal(after[1], before[1])
+            table, lens = _export(lib, pool, R, mb)
+            assert lens.tolist() == length.tolist()
+            assert int(np.sum(table >= 0)) + lib.flide_pool_free_blocks(pool) == n_blocks
+    finally:
+        lib.flide_pool_destroy(pool)
+
+
+def test_store_reserve_is_all_or_nothing():
+    """HistoryStore.reserve (the host half of commit) on CPU buffers: root
+    rows per request, -1 for requests that keep nothing, zero rows for an
+    empty request, and a batch that does not fit changes no slot."""
+    from tree_forked_decision_b200 import inputs
+    from tree_forked_decision_b200.history import HistoryStore
+    store = HistoryStore(n_blocks=5, block_rows=16, max_requests=4, max_blocks=3, Hkv=1, d=8,
+                         device="cpu")
+    tree = inputs._tree([(0, [(-1, 20), (0, 3)]), (0, []), (0, [(-1, 7)]), (0, [(-1, 5), (0, 1)])], 1)
+    start = store.reserve([2, 0, -1, 2], tree)
+    assert start.tolist() == [0, 0, -1, 20]
+    assert store.len_h.tolist() == [0, 0, 25, 0] and store.lengths.tolist() == [0, 0, 25, 0]
+    assert store.free_blocks() == 3
+    assert store.table.tolist() == store.table_h.tolist()
+    with pytest.raises(flide.FlideError) as e:          # 48 + 16 rows: 4 more blocks, 3 free
+        store.reserve([1, 3, -1, -1], inputs._tree([(0, [(-1, 48)]), (0, [(-1, 16)]),
+                                                     (0, [(-1, 1)]), (0, [(-1, 1)])], 0))
+    assert e.value.code == flide.ERR_CAPACITY
+    assert store.len_h.tolist() == [0, 0, 25, 0] and store.free_blocks() == 3

@@ -25,6 +25,7 @@ struct flide_pool {
   std::vector<int32_t> length;   // rows held per request
   std::vector<int32_t> nblocks;  // blocks held per request
   std::vector<int32_t> free_list;
+  std::vector<int64_t> pending;  // per request: rows a batch append adds (0 between calls)
 };
 
 namespace flide {
@@ -184,6 +185,7 @@ flide_pool *flide_pool_create(int32_t n_blocks, int32_t block_rows, int32_t max_
     p->table.assign((size_t)max_requests * max_blocks_per_request, -1);
     p->length.assign(max_requests, 0);
     p->nblocks.assign(max_requests, 0);
+    p->pending.assign(max_requests, 0);
     p->free_list.resize(n_blocks);
     for (int32_t b = 0; b < n_blocks; ++b) p->free_list[b] = n_blocks - 1 - b;  // handed out 0, 1, ...
   } catch (...) {
@@ -199,7 +201,7 @@ int64_t flide_pool_append(flide_pool *p, int32_t slot, int32_t n) {
   if (!p || slot < 0 || slot >= p->max_requests || n < 0) return -FLIDE_ERR_INVALID;
   const int64_t start = p->length[slot];
   const int64_t need = (start + n + p->block_rows - 1) / p->block_rows;
-  if (need > p->max_blocks) return -FLIDE_ERR_CAPACITY;
+  if (need > p->max_blocks || start + n > INT32_MAX) return -FLIDE_ERR_CAPACITY;
   if (need - p->nblocks[slot] > (int64_t)p->free_list.size()) return -FLIDE_ERR_CAPACITY;
   while (p->nblocks[slot] < need) {
     const int32_t b = p->free_list.back();
@@ -208,6 +210,35 @@ int64_t flide_pool_append(flide_pool *p, int32_t slot, int32_t n) {
   }
   p->length[slot] = (int32_t)(start + n);
   return start;
+}
+
+int flide_pool_append_batch(flide_pool *p, int32_t n, const int32_t *slots, const int32_t *counts,
+                            int32_t *starts) {
+  if (!p || n < 0 || (n > 0 && (!slots || !counts || !starts))) return FLIDE_ERR_SHAPE;
+  for (int32_t i = 0; i < n; ++i)
+    if (slots[i] >= p->max_requests || (slots[i] >= 0 && counts[i] < 0)) return FLIDE_ERR_INVALID;
+  // check the whole batch before any reservation: per request the rows it
+  // gains (a request may appear more than once), then its block need
+  for (int32_t i = 0; i < n; ++i)
+    if (slots[i] >= 0) p->pending[slots[i]] += counts[i];
+  int status = FLIDE_OK;
+  int64_t blocks = 0;
+  for (int32_t i = 0; i < n && status == FLIDE_OK; ++i) {
+    const int32_t s = slots[i];
+    if (s < 0 || p->pending[s] < 0) continue;  // skipped, or counted already (marked negative)
+    const int64_t len = (int64_t)p->length[s] + p->pending[s];
+    const int64_t need = (len + p->block_rows - 1) / p->block_rows;
+    if (need > p->max_blocks || len > INT32_MAX) status = FLIDE_ERR_CAPACITY;
+    blocks += need - p->nblocks[s];
+    p->pending[s] = -1 - p->pending[s];
+  }
+  if (status == FLIDE_OK && blocks > (int64_t)p->free_list.size()) status = FLIDE_ERR_CAPACITY;
+  for (int32_t i = 0; i < n; ++i)
+    if (slots[i] >= 0) p->pending[slots[i]] = 0;
+  if (status != FLIDE_OK) return status;
+  for (int32_t i = 0; i < n; ++i)  // cannot fail now
+    starts[i] = slots[i] < 0 ? -1 : (int32_t)flide_pool_append(p, slots[i], counts[i]);
+  return FLIDE_OK;
 }
 
 int flide_pool_release(flide_pool *p, int32_t slot) {

@@ -34,7 +34,8 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_pool_release", "flide_pool_length", "flide_pool_free_blocks", "flide_pool_export",
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
            "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_fork_attn_paged",
-           "flide_plan_state_groups", "flide_copy_rows", "flide_fork_gdn_fp8", "flide_strerror"]
+           "flide_plan_state_groups", "flide_copy_rows", "flide_fork_gdn_fp8", "flide_pool_append_batch",
+           "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -100,6 +101,8 @@ def _lib():
         lib.flide_pool_destroy.restype = None
         lib.flide_pool_append.argtypes = [P, I32, I32]
         lib.flide_pool_append.restype = ctypes.c_int64
+        lib.flide_pool_append_batch.argtypes = [P, I32, P, P, P]
+        lib.flide_pool_append_batch.restype = ctypes.c_int
         lib.flide_pool_release.argtypes = [P, I32]
         lib.flide_pool_release.restype = ctypes.c_int
         lib.flide_pool_length.argtypes = [P, I32]

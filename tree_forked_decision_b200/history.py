@@ -131,20 +131,28 @@ class HistoryStore:
         return flide.fork_attn_paged(q, k, v, index, scale, self.pool_k, self.pool_v, self.table,
                                      req, self.block_rows, self.max_blocks, out=out)
 
+    def reserve(self, slots, tree):
+        """Host half of commit: reserves each request's root rows in its slot
+        (all requests or none: on FlideError no slot changes), refreshes the
+        device block table and lengths, and returns the start rows (-1 where
+        slots[r] is -1)."""
+        slots = [int(s) for s in slots]
+        rp, _parent, seg, _past = tree.arrays()
+        counts = np.array([int(seg[rp[r]]) if rp[r + 1] > rp[r] else 0 for r in range(len(slots))],
+                          np.int32)
+        sl = np.array(slots, np.int32)
+        start = np.zeros(len(slots), np.int32)
+        p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+        flide._check(self._lib.flide_pool_append_batch(self._pool, len(slots), p(sl), p(counts),
+                                                       p(start)), "flide_pool_append_batch")
+        self._sync_table()
+        return start
+
     def commit(self, slots, tree, index: flide.TreeIndex, k, v, node_state=None):
         """Appends request r's root tokens (this step's observation) and its
         root's end GDN state to slot slots[r] (-1: nothing kept)."""
         slots = [int(s) for s in slots]
-        rp, _parent, seg, _past = tree.arrays()
-        start = np.zeros(len(slots), np.int32)
-        for r, s in enumerate(slots):
-            if s < 0 or rp[r + 1] <= rp[r]:
-                continue
-            st = int(self._lib.flide_pool_append(self._pool, s, int(seg[rp[r]])))
-            if st < 0:
-                raise flide.FlideError(-st, "flide_pool_append")
-            start[r] = st
-        self._sync_table()
+        start = self.reserve(slots, tree)
         req = torch.tensor(slots, dtype=torch.int32, device=self.device)
         st_d = torch.from_numpy(start).to(self.device)
         flide._check(self._lib.flide_history_append(
