@@ -238,3 +238,20 @@ def test_selftest_wait_refusals(lib):
     assert lib.flide_selftest_wait_timeout(NUL, 1000, 1, NUL) == S
     assert lib.flide_selftest_wait_timeout(A, 0, 1, NUL) == S
     assert lib.flide_selftest_wait_timeout(A, 10000001, 1, NUL) == S  # waits are bounded at 10 s
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """The binding hands only dense device arrays to the library: a strided
+    view or a host tensor raises before any call."""
+    x = torch.zeros(8, 4, 16)
+    with pytest.raises(ValueError, match="contiguous"):
+        flide._ptr(x.transpose(0, 1))
+    with pytest.raises(ValueError, match="CUDA"):
+        flide._ptr(x)
+    assert flide._ptr(None) is None
+    idx = object.__new__(flide.TreeIndex)
+    with pytest.raises(ValueError, match="CUDA"):
+        flide.fork_attn(torch.zeros(8, 4, 16, dtype=torch.bfloat16),
+                        torch.zeros(8, 2, 16, dtype=torch.bfloat16),
+                        torch.zeros(8, 2, 16, dtype=torch.bfloat16), idx, 0.25,
+                        out=torch.zeros(8, 4, 16, dtype=torch.bfloat16))

@@ -151,7 +151,17 @@ def _check(code, where):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor for the C ABI.  The kernels index dense
+    row-major device arrays, so a strided view or a host tensor is refused
+    here (a host address handed to a kernel would fault the GPU)."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got strides {tuple(t.stride())} "
+                         f"for shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream=None):
