@@ -30,6 +30,11 @@
  *     (malformed tree, capacity overflow) are written to the index's `status`
  *     word (first error wins); kernels that find a non-zero status do nothing.
  *     Read it after synchronising the stream.  No call aborts the process.
+ *   - Host threads: calls may come from several threads at once (the cached
+ *     function pointers and per-device set-up flags are atomic).  Device data
+ *     that calls share (an index and its scratch, the no-alloc work array) is
+ *     ordered by the caller's streams and events, as for any CUDA work.  A
+ *     flide_pool is host state without a lock: one thread at a time.
  *   - Stream layout: requests in order; within a request, nodes in index order
  *     with parent[i] < i; node 0 of each request is its root (the shared
  *     prefix).  Tensors are row-major [token, head, dim].

@@ -606,14 +606,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};  // host threads may race on a first call
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (!fn) {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = (EncodeTiledFn)ptr;
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -665,15 +668,15 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
 
   // the shared-memory opt-in is per device and kernel; remember it for the
   // first 64 devices
-  static bool attr_set[2][64] = {};
+  static std::atomic<bool> attr_set[2][64];  // zero-initialised: false
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLIDE_ERR_CUDA;
-  if (dev < 0 || dev >= 64 || !attr_set[f8][dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[f8][dev].load(std::memory_order_acquire)) {
     const cudaError_t e =
         f8 ? cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
            : cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return FLIDE_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[f8][dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[f8][dev].store(true, std::memory_order_release);
   }
   attn_items_kernel<<<1, 1024, 0, s>>>(*x, Hkv, 2 * mtok);
   FLIDE_LAUNCH_CHECK();
@@ -723,13 +726,16 @@ static __device__ __align__(256) int32_t g_noalloc_work[kNoAllocMaxRequests + 1]
 // array's name only stands in for the symbol, so the address is looked up once
 // per device with that device current and cached.
 int32_t *noalloc_work_ptr() {
-  static int32_t *cached[64] = {};
+  static std::atomic<int32_t *> cached[64];  // zero-initialised: null
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  if (dev >= 0 && dev < 64) {
+    int32_t *c = cached[dev].load(std::memory_order_acquire);
+    if (c) return c;
+  }
   void *p = nullptr;
   if (cudaGetSymbolAddress(&p, g_noalloc_work) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64) cached[dev] = (int32_t *)p;
+  if (dev >= 0 && dev < 64) cached[dev].store((int32_t *)p, std::memory_order_release);
   return (int32_t *)p;
 }
 

@@ -1,6 +1,8 @@
 // common.cuh -- small device helpers shared by the flide kernels.
 #pragma once
 
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>

@@ -335,14 +335,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn_lp() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};  // host threads may race on a first call
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (!fn) {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = (EncodeTiledFn)ptr;
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -399,12 +402,12 @@ extern "C" int flide_branch_logprob(const void *h, const void *w_lm, const int32
 
   CUtensorMap mh, mw;
   if (!make_map_2d(&mh, h, idx->T, D) || !make_map_2d(&mw, w_lm, V, D)) return FLIDE_ERR_CUDA;
-  static bool attr_set[64] = {};
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(branch_logprob_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES) != cudaSuccess)
       return FLIDE_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
   const int tbl = idx->R + 1;  // work[R+1 .. 2R+2): per-request row-tile table
   lp_items_kernel<<<1, 1024, 0, s>>>(*idx, tbl);

@@ -831,14 +831,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn_gdn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};  // host threads may race on a first call
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (!fn) {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = (EncodeTiledFn)ptr;
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -876,15 +879,15 @@ int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, con
   if (!make_map_gdn(&mq, q, H, T, esz) || !make_map_gdn(&mk, k, H, T, esz) ||
       !make_map_gdn(&mv, v, H, T, esz))
     return FLIDE_ERR_CUDA;
-  static bool attr_set[2][64] = {};
+  static std::atomic<bool> attr_set[2][64];  // zero-initialised: false
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLIDE_ERR_CUDA;
-  if (dev < 0 || dev >= 64 || !attr_set[f8][dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[f8][dev].load(std::memory_order_acquire)) {
     const cudaError_t e =
         f8 ? cudaFuncSetAttribute(gdn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
            : cudaFuncSetAttribute(gdn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return FLIDE_ERR_CUDA;
-    if (dev >= 0 && dev < 64) attr_set[f8][dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[f8][dev].store(true, std::memory_order_release);
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
