@@ -98,3 +98,17 @@ def test_tvd_special_cases():
     q[[1, 2]] = 0.5
     q[[5, 6, 7]] = 1.0 / 3
     assert np.allclose(oracle.tvd(t.arrays(), p, q), [0.5, 2.0 / 3])
+
+
+def test_tvd_equals_largest_event_difference():
+    """TVD is also the largest |P(A) - Q(A)| over events A: checked by
+    enumerating every subset of a request's leaves."""
+    import itertools
+    t = inputs._tree([(0, [(-1, 2), (0, 1), (0, 1), (0, 1), (0, 1)])], 1)
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        p, q = np.zeros(t.N), np.zeros(t.N)
+        p[1:], q[1:] = rng.dirichlet(np.ones(4)), rng.dirichlet(np.ones(4))
+        sup = max(abs(p[list(A)].sum() - q[list(A)].sum())
+                  for k in range(5) for A in itertools.combinations(range(1, 5), k))
+        assert math.isclose(oracle.tvd(t.arrays(), p, q)[0], sup, rel_tol=1e-12, abs_tol=1e-15)

@@ -194,3 +194,60 @@ def test_fp8_input_generators_emit_no_nan_codes():
         assert c.dtype == np.uint8 and not np.any((c & 0x7F) == 0x7F)
     assert a["q"].shape == (tree.T, 4, 16) and a["past_k"].shape == (tree.P_past, 2, 16)
     assert np.isclose(a["descale"].numpy(), 1 / 400.0).all()
+
+
+def test_every_midpoint_rounds_like_torch():
+    """Each halfway point between neighbouring finite magnitudes (and the
+    points just either side of it) encodes as torch's float8_e4m3fn
+    conversion does: ties go to the even mantissa."""
+    mags = np.unique(np.abs(fp8.decode_e4m3(np.arange(0x7F, dtype=np.uint8))))
+    mid = (mags[:-1] + mags[1:]) / 2
+    pts = np.concatenate([mid, np.nextafter(mid, 0), np.nextafter(mid, np.inf)])
+    pts = np.concatenate([pts, -pts]).astype(np.float32)
+    pts = pts[np.abs(pts) < 448]
+    want = torch.from_numpy(pts).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(fp8.encode_e4m3(pts), want)
+
+
+def test_dequantised_values_round_trip_within_half_a_step():
+    """decode(code) * descale returns x to within half a code step of the
+    scaled value (relative 2^-4 for normals, 2^-10 absolute below), and a
+    value past the tensor's amax saturates to +-448 times descale."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal(3000) * 3.0).astype(np.float32)
+    codes, ds = fp8.quantize_e4m3(x)
+    back = fp8.decode_e4m3(codes) * float(ds)
+    scale = float(ds)
+    tol = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scale) * (1 + 1e-6)
+    assert (np.abs(back - x) <= tol).all()
+    codes2, ds2 = fp8.quantize_e4m3(x * 4, amax=np.abs(x).max())
+    over = np.abs(x * 4) > np.abs(x).max() * (1 + 2.0 ** -3)
+    assert over.any() and np.allclose(np.abs(fp8.decode_e4m3(codes2[over])), 448.0)
+
+
+def test_encode_saturates_and_never_makes_nan():
+    big = np.array([448.0, 449.0, 464.0, 480.0, 1000.0, 3.0e38, np.inf], np.float64)
+    for v in (big, -big):
+        c = fp8.encode_e4m3(v)
+        assert ((c & 0x7F) == 0x7E).all()
+        assert np.array_equal(fp8.decode_e4m3(c), np.sign(v) * 448.0)
+
+
+def test_attention_fp8_two_keys_closed_form():
+    """One request, a root of two tokens: the second query attends to both
+    keys with weights softmax(c sq sk <Q, K_j>) and returns sv times the
+    weighted decoded values -- the descale factors of q, k and v each enter
+    once."""
+    d = 4
+    q8 = fp8.encode_e4m3(np.array([[[1.0, 0.5, 0.0, -1.0]]] * 2))
+    k8 = fp8.encode_e4m3(np.array([[[2.0, 0.0, 1.0, 0.0]], [[0.0, 1.0, -1.0, 2.0]]]))
+    v8 = fp8.encode_e4m3(np.array([[[1.0, 2.0, 3.0, 4.0]], [[-1.0, 0.0, 0.5, 8.0]]]))
+    sq, sk, sv, scale = 0.5, 0.25, 2.0, 1.0 / math.sqrt(d)
+    tree = ([0, 1], [-1], [2], [0])
+    got = fp8.attention_fp8(tree, q8, k8, v8, None, None, (sq, sk, sv), scale)
+    Q, K, V = (fp8.decode_e4m3(a) for a in (q8, k8, v8))
+    s = scale * (sq * Q[1, 0]) @ (sk * K[:, 0]).T
+    w = np.exp(s - s.max())
+    w /= w.sum()
+    np.testing.assert_allclose(got[1, 0], w @ (sv * V[:, 0]), rtol=1e-12)
+    np.testing.assert_allclose(got[0, 0], sv * V[0, 0], rtol=1e-12)   # first token: its own key only
