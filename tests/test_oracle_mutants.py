@@ -13,6 +13,17 @@ method is likely to make:
   erase_without_beta   the delta rule erases S k k^T without beta
   skipped_root         the root's tokens are left out of every branch's keys
   positions_no_past    isolated positions ignore the checkpointed past
+  gqa_modulo           query head h reads kv head h % Hkv instead of h / G
+  depth_counts_nodes   depth counts nodes instead of edges
+  ctx_without_own_node context length leaves out the node's own tokens
+  children_from_request_state  memoised children restart from the request's
+                       state instead of their parent's end state
+  resume_state_ignored a resumed request starts from zero
+  gate_not_exponentiated  the decay uses 1 + g instead of exp(g)
+  read_before_write    o_t reads the state before token t's update
+  erase_sign           the delta rule adds S k k^T instead of erasing it
+
+The child processes run a few at a time, one oracle thread each.
 """
 import os
 import re
@@ -23,6 +34,13 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "flide_oracle.c")
+
+# one token's write and read in the GDN scan (the read must follow the write)
+_STEP = ("            gdn_step(S, dk, dv, k + ((size_t)t * H + h) * dk,\n"
+         "                     v + ((size_t)t * H + h) * dv,\n"
+         "                     (double)g[(size_t)t * H + h],\n"
+         "                     (double)beta[(size_t)t * H + h], u);\n")
+_READ = "            gdn_read(S, dk, dv, q + ((size_t)t * H + h) * dk, o);\n"
 
 MUTANTS = {
     "exclusive_diagonal": ("for (int j = node_start[n]; j <= t; ++j) {",
@@ -37,33 +55,38 @@ MUTANTS = {
                      "  for (int a = 1; a + 1 < cnt; ++a)\n    for (int j = 0; j < seg_len[chain[a]]; ++j) {\n"
                      "      if (m >= cap) return -1;\n      keys[m++] = node_start[chain[a]] + j;"),
     "positions_no_past": ("int before = past_len[r];", "int before = 0;"),
+    "gqa_modulo": ("int kvh = h / G;", "int kvh = h % Hkv;"),
+    "depth_counts_nodes": ("depth[n] = cnt - 1;", "depth[n] = cnt;"),
+    "ctx_without_own_node": ("ctx += seg_len[chain[i]];", "if (i + 1 < cnt) ctx += seg_len[chain[i]];"),
+    "children_from_request_state": ("if (memoise && parent[n] >= 0) {", "if (0) {"),
+    "resume_state_ignored": [("} else if (state_in_f64) {", "} else if (0) {"),
+                             ("} else if (state_in) {", "} else if (0) {")],
+    "gate_not_exponentiated": ("double alpha = exp(g);", "double alpha = 1.0 + g;"),
+    "read_before_write": (_STEP + _READ, _READ + _STEP),
+    "erase_sign": ("alpha * (S[(size_t)i * dk + c] - w * kc)", "alpha * (S[(size_t)i * dk + c] + w * kc)"),
 }
 
 MIN_FAILED = 5
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_planted_mistake_fails_pins(name):
-    old, new = MUTANTS[name]
+def _c_job(name):
+    """Child-process code that runs the pins against a copy of the C oracle
+    with mistake `name` planted (the copy is written and built here)."""
+    edits = MUTANTS[name] if isinstance(MUTANTS[name], list) else [MUTANTS[name]]
     src = open(SRC).read()
-    assert src.count(old) == 1, "the mutation site must be unique"
+    for old, new in edits:
+        assert src.count(old) == 1, "the mutation site must be unique"
+        src = src.replace(old, new)
     d = os.path.join(ROOT, "oracle", "_build", "mutants", name)
     os.makedirs(d, exist_ok=True)
     msrc, mso = os.path.join(d, "flide_oracle.c"), os.path.join(d, "liboracle.so")
     with open(msrc, "w") as f:
-        f.write(src.replace(old, new))
+        f.write(src)
     if os.path.exists(mso):
         os.remove(mso)
-    code = ("import sys, oracle, pytest\n"
+    return ("import sys, oracle, pytest\n"
             f"oracle._SRC = {msrc!r}\noracle._SO = {mso!r}\n"
             "sys.exit(pytest.main(['-q', '-p', 'no:cacheprovider', 'tests/test_oracle_pins.py']))\n")
-    p = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
-                       timeout=600)
-    assert os.path.exists(mso), p.stdout[-2000:] + p.stderr[-2000:]
-    m = re.search(r"(\d+) failed", p.stdout)
-    failed = int(m.group(1)) if m else 0
-    print(f"{name}: {failed} pins failed")
-    assert failed >= MIN_FAILED, p.stdout[-3000:]
 
 
 # The Python oracles (e4m3 and decision scoring): a mistake is planted by
@@ -94,13 +117,11 @@ PY_MUTANTS = {
 PY_MIN_FAILED = 2
 
 
-@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
-def test_planted_mistake_fails_python_oracle_pins(name):
+def _py_job(name):
     mod, pins, old, new = PY_MUTANTS[name]
     path = os.path.join(ROOT, "oracle", f"{mod}.py")
-    src = open(path).read()
-    assert src.count(old) == 1, "the mutation site must be unique"
-    code = ("import sys, pytest, oracle\n"
+    assert open(path).read().count(old) == 1, "the mutation site must be unique"
+    return ("import sys, pytest, oracle\n"
             f"import oracle.{mod} as m\n"
             "orig = dict(m.__dict__)\n"
             f"src = open({path!r}).read().replace({old!r}, {new!r})\n"
@@ -109,9 +130,45 @@ def test_planted_mistake_fails_python_oracle_pins(name):
             "    if k in orig and orig[k] is v and m.__dict__[k] is not v:\n"
             "        setattr(oracle, k, m.__dict__[k])\n"
             f"sys.exit(pytest.main(['-q', '-p', 'no:cacheprovider', 'tests/{pins}']))\n")
-    p = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
-                       timeout=600)
-    m = re.search(r"(\d+) failed", p.stdout)
-    failed = int(m.group(1)) if m else 0
+
+
+def _run_all(jobs):
+    """Runs the child processes a few at a time (one oracle thread each) and
+    returns per job the number of failed pins and the child's output."""
+    from concurrent.futures import ThreadPoolExecutor
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+
+    def run(code):
+        p = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                           text=True, timeout=600)
+        m = re.search(r"(\d+) failed", p.stdout)
+        return (int(m.group(1)) if m else 0), p.stdout[-3000:] + p.stderr[-2000:]
+
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        futures = {name: ex.submit(run, code) for name, code in jobs.items()}
+        return {name: f.result() for name, f in futures.items()}
+
+
+@pytest.fixture(scope="module")
+def c_runs():
+    return _run_all({name: _c_job(name) for name in MUTANTS})
+
+
+@pytest.fixture(scope="module")
+def py_runs():
+    return _run_all({name: _py_job(name) for name in PY_MUTANTS})
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_pins(name, c_runs):
+    failed, log = c_runs[name]
+    assert os.path.exists(os.path.join(ROOT, "oracle", "_build", "mutants", name, "liboracle.so")), log
     print(f"{name}: {failed} pins failed")
-    assert failed >= PY_MIN_FAILED, p.stdout[-3000:]
+    assert failed >= MIN_FAILED, log
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_planted_mistake_fails_python_oracle_pins(name, py_runs):
+    failed, log = py_runs[name]
+    print(f"{name}: {failed} pins failed")
+    assert failed >= PY_MIN_FAILED, log
