@@ -356,6 +356,12 @@ def percentiles(xs):
     return pick(0.50), pick(0.95)
 
 
+def all_ranks(flag: bool, pg, device) -> bool:
+    """True only if `flag` holds on every rank (a MIN all-reduce), so that legs
+    holding barriers or collectives run on all ranks or on none."""
+    return -max_over_ranks(-float(bool(flag)), pg, device) > 0
+
+
 def job_throughput(units_per_rank: int, steps: int, world: int, ms_max: float) -> float:
     """Whole-job units per second: every rank's units over the slowest rank's time."""
     return units_per_rank * steps * world / (ms_max / 1000.0)
@@ -782,10 +788,10 @@ def main():
         # attention reading the past in place from the blocks, against the same
         # attention over the packed copy
         tree_w, keep = inputs.warm_variant(tree)
-        run_paged = float(tree_w.P_past == rows and a["d"] == 128 and step.q.dtype == torch.bfloat16)
-        if pg is not None:  # the same legs on every rank (they hold barriers)
-            run_paged = -max_over_ranks(-run_paged, pg, device)
-        if run_paged > 0:
+        # the same legs on every rank (they hold barriers)
+        run_paged = all_ranks(tree_w.P_past == rows and a["d"] == 128 and step.q.dtype == torch.bfloat16,
+                              pg, device)
+        if run_paged:
             ridx = torch.from_numpy(keep).to(device)
             qw, kw, vw = (t[ridx].contiguous() for t in (step.q, step.k, step.v))
             dtw = flide.DeviceTree(*tree_w.arrays(), max_depth=max(tree_w.levels, 1), device=device)
@@ -932,10 +938,9 @@ def main():
     bounded = None
     # every rank takes the same legs (each has barriers): the leg runs only if
     # every rank's batch has inner nodes below its roots
-    run_bounded = float(not args.no_bounded and g is not None and flide.state_slots(tree) > tree.R)
-    if pg is not None:
-        run_bounded = -max_over_ranks(-run_bounded, pg, device)
-    if run_bounded > 0:
+    run_bounded = all_ranks(not args.no_bounded and g is not None and flide.state_slots(tree) > tree.R,
+                            pg, device)
+    if run_bounded:
         from tree_forked_decision_b200.schedule import BoundedGdn, plan_state_groups
         full = flide.state_slots(tree)
         budget = max(-(-full // 4), 1)

@@ -4,7 +4,8 @@ The hot path shards by request: each rank serves its own batch and there is no
 data-path collective, so the job's only exchange is the MAX all-reduce of the
 timed region (and of the end-to-end leg).  These tests run that logic in two
 processes: the ranks draw independent batches, both see the slowest rank's
-time, and the whole-job throughput counts every rank's units over that time.
+time, the whole-job throughput counts every rank's units over that time, and
+a leg that holds barriers runs on every rank or on none (a MIN all-reduce).
 """
 import datetime
 import os
@@ -40,8 +41,12 @@ def _rank_main(rank, world, port, out_dir):
         ms_local = 10.0 + 2.5 * r  # this rank's timed region, as if measured
         ms = bench.max_over_ranks(ms_local, dist, "cpu")
         value = bench.job_throughput(tree.branch_tokens, STEPS, ws, ms)
+        # a leg that holds barriers runs on every rank or on none
+        only_rank0 = bench.all_ranks(r == 0, dist, "cpu")
+        everywhere = bench.all_ranks(True, dist, "cpu")
         np.savez(os.path.join(out_dir, f"rank{r}.npz"), ws=ws, seed=seed, q=a["q"].numpy(),
-                 gk=g["k"].numpy(), ms=ms, value=value, branch=tree.branch_tokens)
+                 gk=g["k"].numpy(), ms=ms, value=value, branch=tree.branch_tokens,
+                 only_rank0=only_rank0, everywhere=everywhere)
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -66,6 +71,9 @@ def test_two_ranks_independent_batches_and_max_time(tmp_path):
     expect = units * STEPS / 0.0125
     assert abs(float(r0["value"]) - expect) <= 1e-9 * expect
     assert float(r0["value"]) == float(r1["value"])
+    # leg decisions agree across ranks
+    assert not bool(r0["only_rank0"]) and not bool(r1["only_rank0"])
+    assert bool(r0["everywhere"]) and bool(r1["everywhere"])
 
 
 def test_rank_seed_and_throughput_single_rank():
@@ -74,6 +82,7 @@ def test_rank_seed_and_throughput_single_rank():
     assert bench.rank_seed(WORKLOAD, None, 0) == inputs.WORKLOADS[WORKLOAD]["idx"]
     assert bench.rank_seed(WORKLOAD, 7, 3) == 3007
     assert bench.max_over_ranks(4.25, None, "cpu") == 4.25
+    assert bench.all_ranks(True, None, "cpu") is True and bench.all_ranks(0, None, "cpu") is False
     assert bench.job_throughput(100, 2, 1, 50.0) == 4000.0
     assert bench.percentiles([5.0, 1.0, 2.0, 3.0, 4.0, 6.0, 7.0, 8.0, 9.0, 10.0]) == (5.0, 10.0)
     assert bench.percentiles([2.5]) == (2.5, 2.5)
