@@ -444,7 +444,8 @@ int flide_pool_export(const flide_pool *pool, int32_t *table, int32_t *lengths);
  * its root's end state node_state[state_slot[root]] to pool_S[req_slot[r]]
  * (when node_state and pool_S are given).  start[r] is what flide_pool_append
  * returned (or flide_pool_append_batch wrote).  A row without a block sets
- * FLIDE_ERR_CAPACITY in idx->status.
+ * FLIDE_ERR_CAPACITY in idx->status.  Each slot at most once per call: two
+ * requests of one call writing the same slot's state would race.
  * All arrays are device memory; row bytes (Hkv d element size) % 16 == 0. */
 int flide_history_append(const flide_tree_index *idx, const int32_t *req_slot,
                          const int32_t *start, const int32_t *table, int32_t max_blocks,

@@ -181,13 +181,18 @@ def test_store_reserve_is_all_or_nothing():
     store = HistoryStore(n_blocks=5, block_rows=16, max_requests=4, max_blocks=3, Hkv=1, d=8,
                          device="cpu")
     tree = inputs._tree([(0, [(-1, 20), (0, 3)]), (0, []), (0, [(-1, 7)]), (0, [(-1, 5), (0, 1)])], 1)
-    start = store.reserve([2, 0, -1, 2], tree)
-    assert start.tolist() == [0, 0, -1, 20]
-    assert store.len_h.tolist() == [0, 0, 25, 0] and store.lengths.tolist() == [0, 0, 25, 0]
-    assert store.free_blocks() == 3
+    start = store.reserve([2, 0, -1, 3], tree)
+    assert start.tolist() == [0, 0, -1, 0]
+    assert store.len_h.tolist() == [0, 0, 20, 5] and store.lengths.tolist() == [0, 0, 20, 5]
+    assert store.free_blocks() == 2                     # 2 blocks for slot 2, 1 for slot 3
     assert store.table.tolist() == store.table_h.tolist()
-    with pytest.raises(flide.FlideError) as e:          # 48 + 16 rows: 4 more blocks, 3 free
-        store.reserve([1, 3, -1, -1], inputs._tree([(0, [(-1, 48)]), (0, [(-1, 16)]),
+    start = store.reserve([-1, -1, 3, -1], tree)         # slot 3 continues: 7 more rows
+    assert start.tolist() == [-1, -1, 5, -1] and store.len_h.tolist() == [0, 0, 20, 12]
+    with pytest.raises(flide.FlideError) as e:          # 48 rows: 3 more blocks, 2 free
+        store.reserve([1, 3, -1, -1], inputs._tree([(0, [(-1, 48)]), (0, [(-1, 1)]),
                                                      (0, [(-1, 1)]), (0, [(-1, 1)])], 0))
     assert e.value.code == flide.ERR_CAPACITY
-    assert store.len_h.tolist() == [0, 0, 25, 0] and store.free_blocks() == 3
+    assert store.len_h.tolist() == [0, 0, 20, 12] and store.free_blocks() == 2
+    with pytest.raises(ValueError):                      # one request per slot per step
+        store.reserve([1, 1, -1, -1], tree)
+    assert store.len_h.tolist() == [0, 0, 20, 12]

@@ -135,8 +135,12 @@ class HistoryStore:
         """Host half of commit: reserves each request's root rows in its slot
         (all requests or none: on FlideError no slot changes), refreshes the
         device block table and lengths, and returns the start rows (-1 where
-        slots[r] is -1)."""
+        slots[r] is -1).  Each slot at most once per step (ValueError)."""
         slots = [int(s) for s in slots]
+        kept = [s for s in slots if s >= 0]
+        if len(set(kept)) != len(kept):
+            raise ValueError("a slot may be continued by one request per step "
+                             "(two end states would race for it)")
         rp, _parent, seg, _past = tree.arrays()
         counts = np.array([int(seg[rp[r]]) if rp[r + 1] > rp[r] else 0 for r in range(len(slots))],
                           np.int32)
