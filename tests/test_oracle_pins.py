@@ -437,3 +437,22 @@ def test_gdn_sibling_independence():
     t2 = inputs._tree([(0, [(-1, 5), (0, 3), (1, 2)])], 2)
     o2 = oracle.gdn(t2.arrays(), *(a[x][keep] for x in ("q", "k", "v", "g", "beta")))
     assert np.array_equal(o1[keep], o2)
+
+
+def test_gdn_value_rows_are_independent():
+    """Row i of the state evolves from row i, v_i and the shared k, beta and
+    alpha only (the gated delta rule acts on S from the right), so scanning
+    the two halves of the value dimension separately, each from its half of
+    the initial state, gives the full scan's outputs and end states exactly."""
+    t = inputs.random_tree(np.random.default_rng(31), R=3, max_nodes=6, prefix_range=(2, 12),
+                           branch_range=(1, 6), past_range=(0, 5))
+    a = _rand_gdn(t, 2, 6, 8, 32)
+    S0 = np.random.default_rng(33).standard_normal((t.R, 2, 8, 6))
+    full, st = oracle.gdn(t.arrays(), a["q"], a["k"], a["v"], a["g"], a["beta"], state_in=S0,
+                          want_states=True)
+    for lo, hi in ((0, 3), (3, 8)):
+        part, sp = oracle.gdn(t.arrays(), a["q"], a["k"], np.ascontiguousarray(a["v"][:, :, lo:hi]),
+                              a["g"], a["beta"], state_in=np.ascontiguousarray(S0[:, :, lo:hi]),
+                              want_states=True)
+        np.testing.assert_array_equal(part, full[:, :, lo:hi])
+        np.testing.assert_array_equal(sp, st[:, :, lo:hi])
