@@ -486,8 +486,9 @@ int flide_history_gather(int32_t R, const int32_t *req_slot, int32_t max_request
  * order, packed greedily so that each group's batch needs at most max_slots
  * node-state slots (one per request root in the group, plus its widest odd and
  * widest even depth's inner nodes, as flide_tree_build assigns them).  Returns
- * FLIDE_ERR_CAPACITY if one subtree alone needs more, FLIDE_ERR_INVALID for a
- * malformed tree, FLIDE_ERR_SHAPE for bad arguments. */
+ * FLIDE_ERR_CAPACITY if one subtree alone needs more (or host memory runs
+ * out), FLIDE_ERR_INVALID for a malformed tree (req_node_ptr not starting at
+ * 0 or not monotone, a bad parent), FLIDE_ERR_SHAPE for bad arguments. */
 int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
                             int32_t max_slots, int32_t *node_group, int32_t *n_groups);
 

@@ -97,6 +97,11 @@ def test_refuses_malformed_trees_and_bad_budgets():
     assert lib.flide_plan_state_groups(1, p(rp), p(good), 0, p(out), ctypes.byref(ng)) == flide.ERR_SHAPE
     assert lib.flide_plan_state_groups(1, p(rp), p(good), 1, p(out), ctypes.byref(ng)) == flide.OK
     assert ng.value == 1 and out.tolist() == [-1, 0, 0]
+    # request tables that are not monotone are refused before anything is sized
+    for bad_rp in ([0, -5], [0, 3, 2], [0, 2, -1]):
+        t = np.array(bad_rp, np.int32)
+        assert lib.flide_plan_state_groups(len(t) - 1, p(t), p(good), 4, p(out), ctypes.byref(ng)) \
+            == flide.ERR_INVALID
 
 
 @pytest.mark.parametrize("case", sorted(TREES))
@@ -131,3 +136,50 @@ def test_batches_cover_every_token_row_once(case):
                         if n > brp[bi]:
                             assert 0 <= bpar[n] < n - brp[bi]            # parent precedes
         assert (seen == 1).all()
+
+
+def test_host_entry_points_survive_random_arguments():
+    """Random request tables (monotone or not, negative entries), parents and
+    budgets for the planner, and random slots and counts for the history
+    pool's appends, in a child process: every call returns a status code and
+    the process never aborts (no exception crosses the C ABI)."""
+    import subprocess
+    import sys
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = r'''
+import ctypes, numpy as np
+from tree_forked_decision_b200 import flide
+lib = flide._lib()
+p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+rng = np.random.default_rng(77)
+codes = {flide.OK, flide.ERR_INVALID, flide.ERR_SHAPE, flide.ERR_CAPACITY}
+for _ in range(3000):
+    R = int(rng.integers(0, 6))
+    rp = np.cumsum(np.concatenate([[0], rng.integers(-2, 5, R)])).astype(np.int32)
+    if rng.random() < 0.2:
+        rp[0] = int(rng.integers(-3, 3))
+    N = max(int(rp.max()), 0)
+    parent = rng.integers(-2, 6, max(N, 1)).astype(np.int32)
+    out = np.zeros(max(N, 1), np.int32)
+    ng = ctypes.c_int32(0)
+    st = lib.flide_plan_state_groups(R, p(rp), p(parent), int(rng.integers(-1, 8)), p(out),
+                                     ctypes.byref(ng))
+    assert st in codes, st
+pool = lib.flide_pool_create(12, 4, 5, 3)
+for _ in range(3000):
+    k = int(rng.integers(0, 6))
+    sl = rng.integers(-2, 7, k).astype(np.int32)
+    ct = rng.integers(-3, 20, k).astype(np.int32)
+    starts = np.zeros(max(k, 1), np.int32)
+    st = lib.flide_pool_append_batch(pool, k, p(sl), p(ct), p(starts))
+    assert st in codes, st
+    if rng.random() < 0.3:
+        lib.flide_pool_release(pool, int(rng.integers(-1, 6)))
+    assert 0 <= lib.flide_pool_free_blocks(pool) <= 12
+lib.flide_pool_destroy(pool)
+print("ok")
+'''
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout[-2000:] + r.stderr[-2000:]

@@ -63,12 +63,14 @@ int batch_slots(int roots, const std::vector<int> &inner_at_depth) {
 
 using namespace flide;
 
-extern "C" {
+namespace {
 
-int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
-                            int32_t max_slots, int32_t *node_group, int32_t *n_groups) {
+int plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
+                      int32_t max_slots, int32_t *node_group, int32_t *n_groups) {
   if (R < 0 || !req_node_ptr || !node_group || !n_groups || max_slots < 1) return FLIDE_ERR_SHAPE;
   if (req_node_ptr[0] != 0) return FLIDE_ERR_INVALID;
+  for (int r = 0; r < R; ++r)  // monotone, so N below is a node count
+    if (req_node_ptr[r + 1] < req_node_ptr[r]) return FLIDE_ERR_INVALID;
   const int N = req_node_ptr[R];
   if (N > 0 && !parent) return FLIDE_ERR_SHAPE;
   // per node: depth, level-1 ancestor (global id), whether it has children
@@ -129,6 +131,19 @@ int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_
   }
   *n_groups = g + 1;
   return FLIDE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
+                            int32_t max_slots, int32_t *node_group, int32_t *n_groups) {
+  try {  // no exception may cross the C ABI: out of host memory reads as capacity
+    return plan_state_groups(R, req_node_ptr, parent, max_slots, node_group, n_groups);
+  } catch (...) {
+    return FLIDE_ERR_CAPACITY;
+  }
 }
 
 int flide_copy_rows(void *dst, const void *src, const int32_t *dst_idx, const int32_t *src_idx,
