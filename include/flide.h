@@ -130,7 +130,9 @@ typedef struct {
 } flide_tree_index;
 
 /* Bytes of device memory a tree index with these capacities needs (256-byte
- * aligned sub-arrays).  Returns 0 for negative capacities. */
+ * aligned sub-arrays).  Returns 0 for negative capacities and for capacities
+ * whose arrays would pass 2^31 - 1 entries (the kernels index them with
+ * int32; the ancestor lists take N * (max_depth + 1)). */
 size_t flide_tree_index_bytes(int32_t R, int32_t N, int32_t T, int32_t max_depth);
 
 /* Lays out `idx` over `dev_buf` (device memory of at least `bytes` bytes,

@@ -50,6 +50,12 @@ def test_host_only_entry_points():
     n = lib.flide_tree_index_bytes(4, 30, 1000, 3)
     assert n > 0 and n % 256 == 0
     assert lib.flide_tree_index_bytes(-1, 3, 3, 1) == 0
+    # arrays past int32 indexing are refused (ancestor lists: N * (max_depth + 1))
+    assert lib.flide_tree_index_bytes(1, 2 ** 31 - 1, 10, 2 ** 31 - 1) == 0
+    assert lib.flide_tree_index_bytes(1, 2 ** 20, 10, 2 ** 11) == 0
+    assert lib.flide_tree_index_bytes(1, 2 ** 20, 10, 2 ** 11 - 2) > 0
+    assert lib.flide_tree_index_init(ctypes.byref(flide.TreeIndexC()), ctypes.c_void_p(1 << 20),
+                                     1 << 40, 1, 2 ** 20, 10, 2 ** 11) == flide.ERR_SHAPE
     idx = flide.TreeIndexC()
     # host-only layout over a fake, aligned address: no device access happens
     base = 1 << 20

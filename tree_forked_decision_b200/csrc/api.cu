@@ -59,7 +59,7 @@ bool layout(int32_t R, int32_t N, int32_t T, int32_t D, Layout *L) {
                          N,
                          N,
                          (int64_t)N + 1,
-                         (int64_t)N * (D + 1),
+                         (int64_t)N * ((int64_t)D + 1),
                          N,
                          T,
                          T,
@@ -70,6 +70,9 @@ bool layout(int32_t R, int32_t N, int32_t T, int32_t D, Layout *L) {
                          N,
                          (int64_t)R + 1,
                          work_entries(R, N)};
+  // the kernels index every sub-array with int32
+  for (int i = 0; i < 17; ++i)
+    if (n[i] > INT32_MAX) return false;
   size_t o = 0;
   for (int i = 0; i < 17; ++i) {
     L->off[i] = o;
