@@ -255,3 +255,73 @@ def test_binding_refuses_host_and_strided_tensors():
                         torch.zeros(8, 2, 16, dtype=torch.bfloat16),
                         torch.zeros(8, 2, 16, dtype=torch.bfloat16), idx, 0.25,
                         out=torch.zeros(8, 4, 16, dtype=torch.bfloat16))
+
+
+def test_binding_checks_element_types_and_shapes():
+    """The library reads every tensor of a call as q's element type, so the
+    binding refuses mixed types and inconsistent shapes before any call."""
+    idx = object.__new__(flide.TreeIndex)
+    bf, f32 = torch.bfloat16, torch.float32
+    q, k = torch.zeros(8, 4, 16, dtype=bf), torch.zeros(8, 2, 16, dtype=bf)
+    for fn in (flide.fork_attn, flide.fork_attn_noalloc):
+        with pytest.raises(TypeError, match="k is"):
+            fn(q, k.float(), k, idx, 0.25)
+        with pytest.raises(TypeError, match="out is"):
+            fn(q, k, k, idx, 0.25, out=torch.zeros(8, 4, 16))
+        with pytest.raises(ValueError):
+            fn(q, k, torch.zeros(8, 2, 8, dtype=bf), idx, 0.25)          # v shape
+        with pytest.raises(ValueError):
+            fn(q, torch.zeros(7, 2, 16, dtype=bf), torch.zeros(7, 2, 16, dtype=bf), idx, 0.25)
+        with pytest.raises(ValueError):
+            fn(q, k, k, idx, 0.25, past_k=torch.zeros(3, 1, 16, dtype=bf),
+               past_v=torch.zeros(3, 1, 16, dtype=bf))                   # past heads
+        with pytest.raises(TypeError, match="past_k is"):
+            fn(q, k, k, idx, 0.25, past_k=torch.zeros(3, 2, 16), past_v=torch.zeros(3, 2, 16))
+    gq, gv = torch.zeros(8, 2, 16, dtype=bf), torch.zeros(8, 2, 32, dtype=bf)
+    g = torch.zeros(8, 2, dtype=f32)
+    ns = torch.zeros(3, 2, 32, 16, dtype=f32)
+    with pytest.raises(TypeError, match="g must"):
+        flide.fork_gdn(gq, gq, gv, g.double(), g, idx, ns)
+    with pytest.raises(TypeError, match="node_state"):
+        flide.fork_gdn(gq, gq, gv, g, g, idx, torch.zeros(3, 2, 16, 32, dtype=f32))   # [dv, dk] swapped
+    with pytest.raises(TypeError, match="state_in"):
+        flide.fork_gdn(gq, gq, gv, g, g, idx, ns, state_in=torch.zeros(1, 2, 32, 16, dtype=bf))
+    with pytest.raises(TypeError, match="v is"):
+        flide.fork_gdn(gq, gq, gv.float(), g, g, idx, ns)
+    with pytest.raises(ValueError):
+        flide.fork_gdn(gq, gq, torch.zeros(7, 2, 32, dtype=bf), g, g, idx, ns)
+    # consistent arguments get as far as the device check
+    with pytest.raises(ValueError, match="CUDA"):
+        flide.fork_gdn(gq, gq, gv, g, g, idx, ns, state_in=torch.zeros(1, 2, 32, 16, dtype=f32))
+
+
+def test_binding_checks_paged_and_e4m3_arguments():
+    idx = object.__new__(flide.TreeIndex)
+    bf, u8 = torch.bfloat16, torch.uint8
+    q, k = torch.zeros(8, 4, 128, dtype=bf), torch.zeros(8, 2, 128, dtype=bf)
+    pool = torch.zeros(256, 2, 128, dtype=bf)
+    tab, slot = torch.zeros(4, dtype=torch.int32), torch.zeros(1, dtype=torch.int32)
+    paged = lambda **kw: flide.fork_attn_paged(*[kw.get(n, dflt) for n, dflt in (
+        ("q", q), ("k", k), ("v", k), ("index", idx), ("scale", 0.1), ("pool_k", pool),
+        ("pool_v", pool), ("block_table", tab), ("req_slot", slot), ("block_rows", 128),
+        ("max_blocks", 2))], out=kw.get("out"))
+    with pytest.raises(TypeError, match="pool_k is"):
+        paged(pool_k=pool.float())
+    with pytest.raises(ValueError, match="pools"):
+        paged(pool_v=torch.zeros(256, 1, 128, dtype=bf))
+    with pytest.raises(TypeError, match="block_table"):
+        paged(block_table=tab.long())
+    with pytest.raises(TypeError, match="out must be bfloat16"):
+        paged(out=torch.zeros(8, 4, 128))
+    with pytest.raises(ValueError, match="CUDA"):           # consistent: up to the device check
+        paged()
+    q8, k8 = torch.zeros(8, 4, 128, dtype=u8), torch.zeros(8, 2, 128, dtype=u8)
+    ds = torch.ones(3)
+    with pytest.raises(TypeError, match="out must be bfloat16"):
+        flide.fork_attn_fp8(q8, k8, k8, idx, 0.1, ds, out=torch.zeros(8, 4, 128))
+    g8, g = torch.zeros(8, 2, 128, dtype=u8), torch.zeros(8, 2)
+    ns = torch.zeros(2, 2, 128, 128)
+    with pytest.raises(TypeError, match="beta must"):
+        flide.fork_gdn_fp8(g8, g8, g8, g, g[:, :1].contiguous(), idx, ns, ds)
+    with pytest.raises(TypeError, match="node_state"):
+        flide.fork_gdn_fp8(g8, g8, g8, g, g, idx, torch.zeros(2, 2, 128, 64), ds)

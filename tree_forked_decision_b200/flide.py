@@ -252,6 +252,50 @@ def tree_build(tree: DeviceTree, index: TreeIndex, stream=None):
            "flide_tree_build")
 
 
+
+def _attn_args(where, q, k, v, past_k, past_v, out):
+    """q [T, Hq, d]; k, v [T, Hkv, d]; past_k, past_v [P, Hkv, d]; out like q;
+    one element type for all (the library reads every tensor as q's type)."""
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or k.shape[0] != q.shape[0] \
+            or k.shape[2] != q.shape[2]:
+        raise ValueError(f"{where}: expected q [T, Hq, d] and k, v [T, Hkv, d], got "
+                         f"{tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    for name, t in (("k", k), ("v", v), ("past_k", past_k), ("past_v", past_v), ("out", out)):
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError(f"{where}: {name} is {t.dtype}, q is {q.dtype}")
+    if past_k is not None and past_v is not None and (
+            past_k.shape != past_v.shape or past_k.dim() != 3 or past_k.shape[1:] != k.shape[1:]):
+        raise ValueError(f"{where}: expected past_k, past_v [P, Hkv, d]")
+    if out.shape != q.shape:
+        raise ValueError(f"{where}: out must have q's shape {tuple(q.shape)}")
+
+
+def _bf16_out(where, out, shape):
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != tuple(shape):
+        raise TypeError(f"{where}: out must be bfloat16 {tuple(shape)}")
+
+
+def _gdn_args(where, q, k, v, g, beta, state_in, node_state, out):
+    """q, k [T, H, dk]; v, out [T, H, dv] of q's element type; g, beta [T, H]
+    float32; state_in [R, H, dv, dk] and node_state [slots, H, dv, dk] float32."""
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError(f"{where}: expected q, k [T, H, dk] and v [T, H, dv], got "
+                         f"{tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{where}: {name} is {t.dtype}, q is {q.dtype}")
+    for name, t in (("g", g), ("beta", beta)):
+        if t.dtype != torch.float32 or t.shape != q.shape[:2]:
+            raise TypeError(f"{where}: {name} must be float32 [T, H]")
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    for name, t in (("state_in", state_in), ("node_state", node_state)):
+        if t is not None and (t.dtype != torch.float32 or t.dim() != 4 or tuple(t.shape[1:]) != (H, dv, dk)):
+            raise TypeError(f"{where}: {name} must be float32 [*, {H}, {dv}, {dk}]")
+    if tuple(out.shape) != (T, H, dv):
+        raise ValueError(f"{where}: out must be [{T}, {H}, {dv}]")
+
+
 def fork_attn(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None, out=None,
               flags: int = 0, stream=None):
     T, Hq, d = q.shape
@@ -261,6 +305,7 @@ def fork_attn(q, k, v, index: TreeIndex, scale: float, past_k=None, past_v=None,
     past_rows = 0 if past_k is None else past_k.shape[0]
     if past_rows == 0:
         past_k = past_v = None
+    _attn_args("fork_attn", q, k, v, past_k, past_v, out)
     _check(_lib().flide_fork_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(past_k), _ptr(past_v),
                                   past_rows, ctypes.byref(index.c), Hq, Hkv, d, _dtype_code(q),
                                   float(scale), _ptr(out), flags, _stream(stream)),
@@ -282,6 +327,7 @@ def fork_attn_fp8(q8, k8, v8, index: TreeIndex, scale: float, descale, past_k=No
         raise TypeError("descale must be a float32 tensor of 3 entries")
     if out is None:
         out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    _bf16_out("fork_attn_fp8", out, (T, Hq, d))
     past_rows = 0 if past_k is None else past_k.shape[0]
     if past_rows == 0:
         past_k = past_v = None
@@ -305,6 +351,16 @@ def fork_attn_paged(q, k, v, index: TreeIndex, scale: float, pool_k, pool_v, blo
     dtype = E4M3 if e4m3 else _dtype_code(q)
     if out is None:
         out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _bf16_out("fork_attn_paged", out, (T, Hq, d))
+    byte = lambda t: torch.uint8 if t.dtype == torch.float8_e4m3fn else t.dtype  # e4m3 codes
+    for name, t in (("k", k), ("v", v), ("pool_k", pool_k), ("pool_v", pool_v)):
+        if byte(t) != byte(q):
+            raise TypeError(f"fork_attn_paged: {name} is {t.dtype}, q is {q.dtype}")
+    if pool_v.shape != pool_k.shape or pool_k.dim() != 3 or pool_k.shape[1:] != k.shape[1:]:
+        raise ValueError("fork_attn_paged: pools must be [n_blocks * block_rows, Hkv, d]")
+    for name, t in (("block_table", block_table), ("req_slot", req_slot)):
+        if t.dtype != torch.int32:
+            raise TypeError(f"fork_attn_paged: {name} must be int32")
     n_blocks = pool_k.shape[0] // block_rows
     n_slots = block_table.numel() // max_blocks
     _check(_lib().flide_fork_attn_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(pool_k), _ptr(pool_v),
@@ -330,6 +386,13 @@ def fork_gdn_fp8(q8, k8, v8, g, beta, index: TreeIndex, node_state, descale, sta
         raise TypeError("descale must be a float32 tensor of 3 entries")
     if out is None:
         out = torch.empty((T, H, dv), dtype=torch.bfloat16, device=q8.device)
+    _bf16_out("fork_gdn_fp8", out, (T, H, dv))
+    for name, t in (("g", g), ("beta", beta)):
+        if t.dtype != torch.float32 or t.shape != q8.shape[:2]:
+            raise TypeError(f"fork_gdn_fp8: {name} must be float32 [T, H]")
+    for name, t in (("state_in", state_in), ("node_state", node_state)):
+        if t is not None and (t.dtype != torch.float32 or t.dim() != 4 or tuple(t.shape[1:]) != (H, dv, dk)):
+            raise TypeError(f"fork_gdn_fp8: {name} must be float32 [*, {H}, {dv}, {dk}]")
     _check(_lib().flide_fork_gdn_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(descale), _ptr(g),
                                      _ptr(beta), _ptr(state_in), ctypes.byref(index.c), H, dk, dv,
                                      _ptr(out), _ptr(node_state), node_state.shape[0],
@@ -377,6 +440,7 @@ def fork_attn_noalloc(q, k, v, index: TreeIndex, scale: float, past_k=None, past
     past_rows = 0 if past_k is None else past_k.shape[0]
     if past_rows == 0:
         past_k = past_v = None
+    _attn_args("fork_attn_noalloc", q, k, v, past_k, past_v, out)
     _check(_lib().flide_fork_attn_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(past_k), _ptr(past_v),
                                           past_rows, ctypes.byref(index.c), Hq, Hkv, d,
                                           _dtype_code(q), float(scale), _ptr(out), flags,
@@ -391,6 +455,7 @@ def fork_gdn(q, k, v, g, beta, index: TreeIndex, node_state, state_in=None, out=
     dv = v.shape[2]
     if out is None:
         out = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    _gdn_args("fork_gdn", q, k, v, g, beta, state_in, node_state, out)
     _check(_lib().flide_fork_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
                                  ctypes.byref(index.c), H, dk, dv, _dtype_code(q), _ptr(out),
                                  _ptr(node_state), node_state.shape[0], flags, _stream(stream)),
