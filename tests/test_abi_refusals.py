@@ -325,3 +325,24 @@ def test_binding_checks_paged_and_e4m3_arguments():
         flide.fork_gdn_fp8(g8, g8, g8, g, g[:, :1].contiguous(), idx, ns, ds)
     with pytest.raises(TypeError, match="node_state"):
         flide.fork_gdn_fp8(g8, g8, g8, g, g, idx, torch.zeros(2, 2, 128, 64), ds)
+
+
+def test_binding_checks_checkpoint_arguments():
+    idx = object.__new__(flide.TreeIndex)
+    bf, i32 = torch.bfloat16, torch.int32
+    k = torch.zeros(8, 2, 16, dtype=bf)
+    ns, cS = torch.zeros(3, 2, 4, 8), torch.zeros(1, 2, 4, 8)
+    with pytest.raises(TypeError, match="ckpt_k"):
+        flide.state_save(idx, k, k, torch.zeros(9, 2, 16), torch.zeros(9, 2, 16, dtype=bf), None)
+    with pytest.raises(TypeError, match="past_v"):
+        flide.state_save(idx, k, k, torch.zeros(9, 2, 16, dtype=bf), torch.zeros(9, 2, 16, dtype=bf),
+                         None, past_k=torch.zeros(1, 2, 16, dtype=bf), past_v=torch.zeros(1, 1, 16, dtype=bf))
+    with pytest.raises(TypeError, match="ckpt_S"):
+        flide.state_save(idx, None, None, None, None, torch.zeros(1, 2, 8, 4), node_state=ns)
+    z = lambda n: torch.zeros(n, dtype=i32)
+    with pytest.raises(TypeError, match="src_req"):
+        flide.state_resume(torch.zeros(1, dtype=torch.int64), z(2), k, k, None, z(1), k, k, None, z(1))
+    with pytest.raises(TypeError, match="past_k"):
+        flide.state_resume(z(1), z(2), k, k, None, z(1), torch.zeros(8, 2, 16), k, None, z(1))
+    with pytest.raises(TypeError, match="src_S"):
+        flide.state_resume(z(1), z(2), k, k, torch.zeros(1, 2, 4, 8, dtype=bf), z(1), k, k, cS, z(1))

@@ -463,6 +463,26 @@ def fork_gdn(q, k, v, g, beta, index: TreeIndex, node_state, state_in=None, out=
     return out
 
 
+def _rows_like(where, ref, **named):
+    """K/V row tensors copied with ref's element type and row layout."""
+    for name, t in named.items():
+        if t is not None and (t.dtype != ref.dtype or t.dim() != 3 or t.shape[1:] != ref.shape[1:]):
+            raise TypeError(f"{where}: {name} must be {ref.dtype} [*, {ref.shape[1]}, {ref.shape[2]}]")
+
+
+def _states_like(where, H, dv, dk, **named):
+    for name, t in named.items():
+        if t is not None and (t.dtype != torch.float32 or t.dim() != 4
+                              or tuple(t.shape[1:]) != (H, dv, dk)):
+            raise TypeError(f"{where}: {name} must be float32 [*, {H}, {dv}, {dk}]")
+
+
+def _int32(where, **named):
+    for name, t in named.items():
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError(f"{where}: {name} must be int32")
+
+
 def state_save(index: TreeIndex, k, v, ckpt_k, ckpt_v, ckpt_S, past_k=None, past_v=None,
                node_state=None, stream=None):
     Hkv, d = (k.shape[1], k.shape[2]) if k is not None else (0, 0)
@@ -470,6 +490,10 @@ def state_save(index: TreeIndex, k, v, ckpt_k, ckpt_v, ckpt_S, past_k=None, past
     if node_state is not None:
         _, H, dv, dk = node_state.shape
     dt = _dtype_code(k) if k is not None else BF16
+    if k is not None:
+        _rows_like("state_save", k, v=v, ckpt_k=ckpt_k, ckpt_v=ckpt_v, past_k=past_k, past_v=past_v)
+    if node_state is not None:
+        _states_like("state_save", H, dv, dk, node_state=node_state, ckpt_S=ckpt_S)
     _check(_lib().flide_state_save(ctypes.byref(index.c), _ptr(k), _ptr(v), _ptr(past_k),
                                    _ptr(past_v), Hkv, d, dt, _ptr(node_state), H, dk, dv,
                                    _ptr(ckpt_k), _ptr(ckpt_v), _ptr(ckpt_S),
@@ -485,6 +509,10 @@ def state_resume(src_req, src_ckpt_start, src_k, src_v, src_S, past_len, past_k,
     H = dv = dk = 0
     if state_in is not None:
         _, H, dv, dk = state_in.shape
+        _states_like("state_resume", H, dv, dk, src_S=src_S, state_in=state_in)
+    _rows_like("state_resume", src_k, src_v=src_v, past_k=past_k, past_v=past_v)
+    _int32("state_resume", src_req=src_req, src_ckpt_start=src_ckpt_start, past_len=past_len,
+           status=status)
     _check(_lib().flide_state_resume(R, _ptr(src_req), src_R, _ptr(src_ckpt_start), _ptr(src_k),
                                      _ptr(src_v), _ptr(src_S), Hkv, d, _dtype_code(src_k), H, dk,
                                      dv, _ptr(past_len), _ptr(past_k), _ptr(past_v),
