@@ -346,3 +346,23 @@ def test_binding_checks_checkpoint_arguments():
         flide.state_resume(z(1), z(2), k, k, None, z(1), torch.zeros(8, 2, 16), k, None, z(1))
     with pytest.raises(TypeError, match="src_S"):
         flide.state_resume(z(1), z(2), k, k, torch.zeros(1, 2, 4, 8, dtype=bf), z(1), k, k, cS, z(1))
+
+
+def test_binding_checks_decision_arguments():
+    idx = flide.TreeIndex.__new__(flide.TreeIndex)
+    idx.R, idx.N, idx.T = 1, 3, 8
+    bf = torch.bfloat16
+    h, w = torch.zeros(8, 64, dtype=bf), torch.zeros(128, 64, dtype=bf)
+    y, lp, ws = torch.zeros(8, dtype=torch.int32), torch.zeros(8), torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(TypeError, match="w_lm"):
+        flide.branch_logprob(h, w.float(), y, idx, logp=lp, workspace=ws)
+    with pytest.raises(TypeError, match="w_lm"):
+        flide.branch_logprob(h, torch.zeros(128, 32, dtype=bf), y, idx, logp=lp, workspace=ws)
+    with pytest.raises(TypeError, match="targets"):
+        flide.branch_logprob(h, w, y.long(), idx, logp=lp, workspace=ws)
+    with pytest.raises(ValueError, match="entries"):
+        flide.branch_logprob(h, w, y[:5], idx, logp=lp, workspace=ws)
+    with pytest.raises(TypeError, match="logp must"):
+        flide.option_probs(idx, lp.double(), path_logp=torch.zeros(3), prob=torch.zeros(3))
+    with pytest.raises(ValueError, match="entries"):
+        flide.option_probs(idx, lp, path_logp=torch.zeros(2), prob=torch.zeros(3))

@@ -545,9 +545,14 @@ def branch_logprob(h, w_lm, targets, index: TreeIndex, logp=None, workspace=None
         logp = torch.empty(T, dtype=torch.float32, device=h.device)
     if workspace is None:
         workspace = branch_logprob_workspace(index, V, device=h.device)
+    if w_lm.dtype != h.dtype or w_lm.dim() != 2 or w_lm.shape[1] != D:
+        raise TypeError(f"branch_logprob: w_lm must be {h.dtype} [V, {D}]")
+    _int32("branch_logprob", targets=targets)
+    if targets.numel() < T or logp.dtype != torch.float32 or logp.numel() < T:
+        raise ValueError(f"branch_logprob: targets (int32) and logp (float32) need {T} entries")
     _check(_lib().flide_branch_logprob(_ptr(h), _ptr(w_lm), _ptr(targets), ctypes.byref(index.c), D, V,
                                        _dtype_code(h), _ptr(logp), _ptr(workspace),
-                                       workspace.numel(), _stream(stream)),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)),
            "flide_branch_logprob")
     return logp
 
@@ -560,6 +565,11 @@ def option_probs(index: TreeIndex, logp, path_logp=None, prob=None, stream=None)
         path_logp = torch.empty(max(N, 1), dtype=torch.float32, device=logp.device)
     if prob is None:
         prob = torch.empty(max(N, 1), dtype=torch.float32, device=logp.device)
+    for name, t in (("logp", logp), ("path_logp", path_logp), ("prob", prob)):
+        if t.dtype != torch.float32:
+            raise TypeError(f"option_probs: {name} must be float32")
+    if path_logp.numel() < N or prob.numel() < N:
+        raise ValueError(f"option_probs: path_logp and prob need {N} entries")
     _check(_lib().flide_option_probs(ctypes.byref(index.c), _ptr(logp), _ptr(path_logp), _ptr(prob),
                                      _stream(stream)),
            "flide_option_probs")
