@@ -447,6 +447,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=2000)
     ap.add_argument("--ref-pairs", type=int, default=16)
     args = ap.parse_args()
+    if args.steps < 1 or args.warmup < 0 or args.gpus < 1:
+        ap.error("--steps and --gpus must be at least 1, --warmup at least 0")
     if args.impl == "reference":
         return run_reference(args)
 

@@ -60,3 +60,8 @@ def test_product_arm_needs_a_device():
     assert p.returncode != 0
     assert "CUDA device" in (p.stdout + p.stderr)
     assert not [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_bad_step_counts_are_refused():
+    p = _bench("--impl", "reference", "--workload", "tiny_fp32", "--steps", "0", "--warmup", "3")
+    assert p.returncode == 2 and "--steps" in p.stderr
