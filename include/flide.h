@@ -357,7 +357,9 @@ int flide_state_save(const flide_tree_index *idx, const void *k, const void *v,
  *   src_req [R] int32 (device)
  *   past_k, past_v [past_rows, Hkv, d]; state_in [R, H, dv, dk] fp32
  * Writes FLIDE_ERR_CAPACITY / FLIDE_ERR_INVALID to *status (device int32) if
- * the rows exceed past_rows or src_req is out of range.
+ * the rows exceed past_rows or src_req is out of range.  R <= 4096 (host
+ * error FLIDE_ERR_CAPACITY beyond); host error FLIDE_ERR_SHAPE for NULL
+ * arrays, an unsupported dtype or K/V rows not a multiple of 16 bytes.
  */
 int flide_state_resume(int32_t R, const int32_t *src_req, int32_t src_R,
                        const int32_t *src_ckpt_start, const void *src_k,

@@ -176,8 +176,8 @@ int state_resume(int R, const int32_t *src_req, int src_R, const int32_t *src_st
                  int H, int dk, int dv, int32_t *past_len, void *pk, void *pv,
                  int past_rows, float *state_in, int32_t *status, cudaStream_t s) {
   const int es = dtype == FLIDE_BF16 ? 2 : (dtype == FLIDE_F32 ? 4 : 0);
-  if (!es || R < 0 || R > kMaxResumeR || !src_req || !src_start || !past_len || !status)
-    return FLIDE_ERR_SHAPE;
+  if (!es || R < 0 || !src_req || !src_start || !past_len || !status) return FLIDE_ERR_SHAPE;
+  if (R > kMaxResumeR) return FLIDE_ERR_CAPACITY;  // the kernel's shared offset table
   const long row_bytes = (long)Hkv * d * es;
   if (row_bytes <= 0 || row_bytes % 16 != 0 || !sk || !sv || !pk || !pv) return FLIDE_ERR_SHAPE;
   if (state_in && (!sS || ((long)dk * dv) % 4 != 0 || H <= 0)) return FLIDE_ERR_SHAPE;
