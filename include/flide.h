@@ -379,7 +379,8 @@ int flide_state_resume(int32_t R, const int32_t *src_req, int32_t src_R,
  * and the decision is the softmax over the request's leaves.
  *
  * Bytes of `workspace` that flide_branch_logprob needs for a tree of up to T
- * stream tokens and a vocabulary of V (partial sums of the vocabulary split). */
+ * stream tokens and a vocabulary of V (partial sums of the vocabulary split);
+ * 0 when T or V is not positive. */
 size_t flide_branch_logprob_workspace_bytes(int32_t T, int32_t V);
 
 /* log p_t = h_t . w_{y_t} - logsumexp_v h_t . w_v for every branch token t
@@ -398,7 +399,9 @@ int flide_branch_logprob(const void *h, const void *w_lm, const int32_t *targets
 /* Per node: path_logp[n] = sum of logp over the branch tokens from the root's
  * child down to n (0 for roots); prob[n] = softmax of path_logp over the leaves
  * of n's request for leaves, 0 for other nodes.  logp [T] fp32 (from
- * flide_branch_logprob), path_logp and prob [N] fp32 out (device). */
+ * flide_branch_logprob), path_logp and prob [N] fp32 out (device).  Host
+ * errors: FLIDE_ERR_SHAPE for NULL arguments, FLIDE_ERR_CUDA; nothing is
+ * launched for a batch without requests. */
 int flide_option_probs(const flide_tree_index *idx, const float *logp, float *path_logp,
                        float *prob, flide_stream stream);
 
@@ -433,13 +436,16 @@ int64_t flide_pool_append(flide_pool *pool, int32_t slot, int32_t n);
  * arrays with n > 0.  Host arrays. */
 int flide_pool_append_batch(flide_pool *pool, int32_t n, const int32_t *slots,
                             const int32_t *counts, int32_t *starts);
-/* Returns all blocks of request `slot` to the free list; its length becomes 0. */
+/* Returns all blocks of request `slot` to the free list; its length becomes 0.
+ * FLIDE_ERR_INVALID for a bad slot. */
 int flide_pool_release(flide_pool *pool, int32_t slot);
-/* History rows held by `slot` (negative status for a bad slot). */
+/* History rows held by `slot`; -FLIDE_ERR_INVALID for a bad slot. */
 int32_t flide_pool_length(const flide_pool *pool, int32_t slot);
+/* Blocks on the free list (0 for a NULL pool). */
 int32_t flide_pool_free_blocks(const flide_pool *pool);
 /* Copies the block table [max_requests * max_blocks_per_request] and the
- * lengths [max_requests] into host arrays. */
+ * lengths [max_requests] into caller-owned host arrays of those sizes.
+ * FLIDE_ERR_SHAPE for NULL arguments. */
 int flide_pool_export(const flide_pool *pool, int32_t *table, int32_t *lengths);
 
 /* After a step: request r of the batch (req_slot[r] >= 0) writes its root's
@@ -516,7 +522,8 @@ int flide_copy_rows(void *dst, const void *src, const int32_t *dst_idx, const in
 int flide_selftest_wait_timeout(int32_t *status, int32_t timeout_us, int32_t arrive,
                                 flide_stream stream);
 
-/* Static message for a status code. */
+/* Static message for a status code ("unknown status" for any other value);
+ * never NULL, owned by the library. */
 const char *flide_strerror(int32_t code);
 
 #ifdef __cplusplus
