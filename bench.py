@@ -423,6 +423,52 @@ def run_reference(args):
     return 0
 
 
+def measure_workload(name, rank, steps, device, pg, local_rank, peak_tflops, hbm_gbs):
+    """A few timed steps of another named workload (same call sequence as the
+    headline step, rank-seeded batch): ms per step, branch-token evals/s and
+    each layer's fraction of its roofline, with the clocks seen meanwhile."""
+    tree, a, g, _ = inputs.make_inputs(name, seed=rank_seed(name, None, rank))
+    st = Step(tree, a, g, device)
+    for _ in range(3):
+        st.run()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(steps):
+            evs[i][3].record()
+            st.run(evs[i])
+            evs[i][4].record()
+        torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    if st.idx.status() != 0:
+        raise SystemExit(f"device status {st.idx.status()} in the {name} timing")
+    ws = pg.get_world_size() if pg is not None else 1
+    step_ms = max_over_ranks(statistics.mean(e[3].elapsed_time(e[4]) for e in evs), pg, device)
+    res = {"ms_per_step": step_ms, "value": job_throughput(tree.branch_tokens, 1, ws, step_ms),
+           "unit": UNIT, "steps": steps, "warmup": 3, "requests_per_gpu": tree.R,
+           "tokens_per_gpu": tree.T, "branch_tokens_per_gpu": tree.branch_tokens,
+           "clocks": clk.summary()}
+    if a is not None:
+        ams = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in evs), pg, device)
+        flops, _ = attn_work(tree, a)
+        tf = flops / (ams / 1000.0) / 1e12
+        res["fork_attn"] = {"ms": ams, "tflops": tf, "frac": tf / peak_tflops, "bound": "tensor",
+                            "algorithmic_flops": flops}
+    if g is not None:
+        gms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in evs), pg, device)
+        gb = gdn_work(tree, g)
+        gbs = gb / (gms / 1000.0) / 1e9
+        res["fork_gdn"] = {"ms": gms, "gbs": gbs, "frac": gbs / hbm_gbs, "bound": "hbm",
+                           "algorithmic_bytes": gb}
+    del st
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -441,6 +487,10 @@ def main():
     ap.add_argument("--no-history", action="store_true", help="skip the paged history store timing")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 attention timing")
     ap.add_argument("--no-bounded", action="store_true", help="skip the memory-bounded GDN timing")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the short timings of the other bf16 workloads")
+    ap.add_argument("--workload-steps", type=int, default=10,
+                    help="timed steps per extra workload (after 3 warm-up steps)")
     ap.add_argument("--vocab", type=int, default=8192, help="LM-head vocabulary of the decision leg")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--cpu-pairs", type=int, default=16)
@@ -684,13 +734,13 @@ def main():
     peaks, peak_src = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    kernels, roofline = {}, None
+    kernels, roofline, roofline_gdn = {}, None, None
     if g is not None:
         gbytes = gdn_work(tree, g)
         gdn_gbs = gbytes / (gdn_ms / 1000.0) / 1e9
         kernels["fork_gdn"] = {"ms": gdn_ms, "algorithmic_bytes": gbytes, "gbs": gdn_gbs,
                                "frac_of_hbm_peak": gdn_gbs / hbm, "bound": "hbm"}
-        roofline = {
+        roofline_gdn = roofline = {
             "kernel": "gdn_tc_kernel (GDN fork scan, tcgen05)", "bound": "hbm", "achieved": gdn_gbs,
             "peak": hbm, "unit": "GB/s", "frac": gdn_gbs / hbm,
             "traffic": traffic_for("gdn_tc_kernel", "gdn_tc.cu"),
@@ -993,6 +1043,18 @@ def main():
         combined = {"roofline_ms": rt, "measured_p50_ms": p50_ms, "frac": rt / p50_ms, "parts": parts,
                     "peaks": "attention: sustained dense bf16; GDN: HBM copy (measured)"}
 
+    # the other bf16 workloads, a few timed steps each (their tree shapes and
+    # head counts differ from the headline one: attention-only fan-out, GDN-only
+    # fan-out, and the mixed hybrid batch of depth 1-3 trees with resumed requests)
+    workloads = None
+    if not args.no_workloads and args.layers == "both":
+        workloads = {}
+        for name in ("attn_fanout_bf16", "gdn_fanout_bf16", "mixed_hybrid_bf16"):
+            if name == args.workload:
+                continue
+            workloads[name] = measure_workload(name, rank, args.workload_steps, device, pg,
+                                               local_rank, peak, hbm)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, desc, threads = cpu_oracle_rate(tree, a, g, args.cpu_rows, args.cpu_pairs)
@@ -1011,7 +1073,9 @@ def main():
                    "l2": "inputs larger than L2 (GBs per step), no flush",
                    "parallelism": f"dp{ws} (independent requests per rank)", "seed": seed},
         "roofline": roofline,
+        "roofline_gdn": roofline_gdn,
         "roofline_combined": combined,
+        "workloads": workloads,
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -502,6 +502,22 @@ int flide_history_gather(int32_t R, const int32_t *req_slot, int32_t max_request
 int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
                             int32_t max_slots, int32_t *node_group, int32_t *n_groups);
 
+/* Host query: the node-state slots flide_tree_build will assign to this batch
+ * (what it writes to counts[FLIDE_CNT_SLOTS]), for sizing the node_state
+ * buffer of flide_fork_gdn before any device work.  One slot per non-empty
+ * request's root (its end state is the request's checkpoint), plus the
+ * largest number of inner nodes (nodes with children) at any odd depth and at
+ * any even depth >= 2: depth L's inner nodes share their region with depth
+ * L + 2, which the scan writes only after depth L + 1 has read them
+ * (techfi24.com, "Limites et perspectives": memory for cloned states is the
+ * limit).  req_node_ptr [R+1] and parent [N] are HOST arrays laid out as in
+ * flide_tree_desc.  Writes *slots and returns FLIDE_OK, FLIDE_ERR_INVALID for
+ * a malformed tree (req_node_ptr not starting at 0 or not monotone, a bad
+ * parent), FLIDE_ERR_SHAPE for a NULL argument or R < 0, FLIDE_ERR_CAPACITY
+ * if host memory runs out. */
+int flide_tree_state_slots(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
+                           int32_t *slots);
+
 /* Device row copy: dst row dst_idx[i] <- src row src_idx[i] for i < n (a NULL
  * index array means i), rows of row_bytes bytes (a multiple of 4; pointers
  * 4-byte aligned, 16-byte words when rows and pointers allow).  Index arrays

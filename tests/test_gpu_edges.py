@@ -8,7 +8,7 @@ import torch
 import oracle
 from tree_forked_decision_b200 import flide, inputs
 
-from gpu_helpers import (assert_close, build, oracle_attn, oracle_gdn, run_attn, run_gdn)
+from gpu_helpers import (assert_close, build, oracle_attn, oracle_gdn, run_attn, run_gdn, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -171,3 +171,47 @@ def test_resume_fresh_request_and_bad_source():
                        sk, sk, sS, past_len, pk, pk.clone(), st, status)
     torch.cuda.synchronize()
     assert int(status.item()) == flide.ERR_INVALID
+
+
+@pytest.mark.parametrize("path", ["tc", "portable", "noalloc"])
+def test_past_buffers_shorter_than_tree_past_are_refused(path):
+    """The tree asks for 80 past rows but the caller passes buffers of 60: the
+    kernels must report FLIDE_ERR_CAPACITY instead of reading rows beyond the
+    buffers (the tensor-core path would otherwise attend to zero rows).  The
+    60-row buffers are views of longer tensors, so no read can leave device
+    memory whatever the kernels do."""
+    tree = inputs._tree([(50, [(-1, 10), (0, 5)]), (30, [(-1, 8), (0, 3)])], 1)
+    rng = np.random.default_rng(9)
+    a = inputs.attn_inputs(tree, 8, 2, 128, torch.bfloat16, rng)
+    assert a["past_k"].shape[0] == 80
+    pk, pv = to_dev(a["past_k"]), to_dev(a["past_v"])
+    _, idx = build(tree)
+    q, k, v = to_dev(a["q"]), to_dev(a["k"]), to_dev(a["v"])
+    if path == "noalloc":
+        flide.fork_attn_noalloc(q, k, v, idx, 0.1, past_k=pk[:60], past_v=pv[:60])
+    else:
+        flags = flide.FLAG_PORTABLE if path == "portable" else 0
+        flide.fork_attn(q, k, v, idx, 0.1, past_k=pk[:60], past_v=pv[:60], flags=flags)
+    torch.cuda.synchronize()
+    assert idx.status() == flide.ERR_CAPACITY
+    # the same call with every row present runs clean
+    _, idx2 = build(tree)
+    flide.fork_attn(q, k, v, idx2, 0.1, past_k=pk, past_v=pv)
+    torch.cuda.synchronize()
+    assert idx2.status() == 0
+
+
+def test_tree_token_total_beyond_int32_is_refused():
+    """Per-node lengths that pass every single check but add up past 2^31 - 1
+    (tokens plus past rows) must give FLIDE_ERR_CAPACITY before the int32
+    prefix sums can wrap.  The descriptor's token capacity is set high so
+    that only the 64-bit total check can catch it; no layer kernel runs."""
+    rp = np.array([0, 3, 5], np.int32)
+    parent = np.array([-1, 0, 0, -1, 0], np.int32)
+    seg = np.array([1, 1, 1, 1, 1], np.int32)
+    past = np.array([0x7ffffff0, 0x20], np.int32)
+    dt = flide.DeviceTree(rp, parent, seg, past, max_depth=1, N=5, T=16)
+    idx = flide.TreeIndex(dt.R, dt.N, dt.T, 1)
+    flide.tree_build(dt, idx)
+    torch.cuda.synchronize()
+    assert idx.status() == flide.ERR_CAPACITY

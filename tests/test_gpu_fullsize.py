@@ -1,8 +1,10 @@
 """Full-size workloads through the C ABI in the launch configuration bench.py
 times, checked against the oracle on sampled outputs: attention on a seeded
 sample of query rows (first and last root rows of every request, every branch
-row of query head 0, plus random rows), GDN on every token of sampled
-(request, head) pairs."""
+row of query head 0, every branch row of the last request for all G query
+heads of the last kv group -- so the in-group positions 1..G-1 of the 128-row
+tile packing are all covered at full size -- plus random rows), GDN on every
+token of sampled (request, head) pairs."""
 import numpy as np
 import pytest
 
@@ -14,10 +16,14 @@ from gpu_helpers import assert_close, run_attn, run_gdn
 pytestmark = pytest.mark.gpu
 
 
-def _rows(tree, Hq, n_random, rng):
+def _rows(tree, Hq, Hkv, n_random, rng):
     starts = np.concatenate([[0], np.cumsum(tree.seg_len)])
     rp = tree.req_node_ptr
     rows = []
+    G = Hq // Hkv
+    last = max(r for r in range(tree.R) if rp[r + 1] > rp[r])
+    for t in range(starts[rp[last] + 1], starts[rp[last + 1]]):  # all heads of kv group Hkv - 1
+        rows += [(t, h) for h in range(Hq - G, Hq)]
     for r in range(tree.R):
         if rp[r + 1] == rp[r]:
             continue
@@ -35,7 +41,7 @@ def test_fullsize_attention_sampled(name):
     tree, a, _, dtype = inputs.make_inputs(name)
     got, scale = run_attn(tree, a)
     rng = np.random.default_rng(1)
-    rows = _rows(tree, a["Hq"], 1500, rng)
+    rows = _rows(tree, a["Hq"], a["Hkv"], 1500, rng)
     f = lambda t: t.float().numpy()
     want = oracle.attention_rows(tree.arrays(), f(a["q"]), f(a["k"]), f(a["v"]),
                                  f(a["past_k"]), f(a["past_v"]), scale, rows)

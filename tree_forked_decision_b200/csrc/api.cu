@@ -10,8 +10,8 @@
 namespace flide {
 int tree_build(const flide_tree_desc *d, flide_tree_index *x, cudaStream_t s);
 int fork_attn_portable(const void *q, const void *k, const void *v, const void *pk,
-                       const void *pv, const flide_tree_index *x, int Hq, int Hkv, int d,
-                       int dtype, float scale, void *out, cudaStream_t s);
+                       const void *pv, int past_rows, const flide_tree_index *x, int Hq,
+                       int Hkv, int d, int dtype, float scale, void *out, cudaStream_t s);
 bool fork_attn_tc_supported(const flide_tree_index *x, int Hq, int Hkv, int d, int dtype);
 int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, const void *pv,
                  int past_rows, const flide_tree_index *x, int Hq, int Hkv, int dtype,
@@ -133,8 +133,8 @@ int flide_fork_attn(const void *q, const void *k, const void *v, const void *pas
   if (!(flags & FLIDE_FLAG_PORTABLE) && fork_attn_tc_supported(idx, Hq, Hkv, d, dtype))
     return fork_attn_tc(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, dtype, nullptr, scale,
                         out, (cudaStream_t)stream, nullptr);
-  return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,
-                            (cudaStream_t)stream);
+  return fork_attn_portable(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, d, dtype, scale,
+                            out, (cudaStream_t)stream);
 }
 
 int flide_fork_attn_fp8(const void *q, const void *k, const void *v, const void *past_k,

@@ -25,7 +25,8 @@ struct PortableArgs {
   T *out;
   flide_tree_index x;
   int Hq, Hkv, d;
-  float qscale;  // scale * log2(e)
+  int past_rows;  // rows of the packed past buffers
+  float qscale;   // scale * log2(e)
 };
 
 template <typename T>
@@ -94,6 +95,10 @@ attn_portable_kernel(PortableArgs<T> a) {
         set_status(x.status, FLIDE_ERR_SHAPE);
         continue;
       }
+      if (p0 < 0 || (long)p0 + plen > a.past_rows) {  // past buffers shorter than the tree's past
+        set_status(x.status, FLIDE_ERR_CAPACITY);
+        continue;
+      }
       attend_span(a, a.pk, a.pv, p0, plen, kvh, qs, m, l, acc);
     }
     // 2. strict ancestors, root first
@@ -116,12 +121,13 @@ attn_portable_kernel(PortableArgs<T> a) {
 
 template <typename T>
 int launch(const void *q, const void *k, const void *v, const void *pk, const void *pv,
-           const flide_tree_index *x, int Hq, int Hkv, int d, float scale, void *out,
-           cudaStream_t s) {
+           int past_rows, const flide_tree_index *x, int Hq, int Hkv, int d, float scale,
+           void *out, cudaStream_t s) {
   PortableArgs<T> a;
   a.q = (const T *)q; a.k = (const T *)k; a.v = (const T *)v;
   a.pk = (const T *)pk; a.pv = (const T *)pv; a.out = (T *)out;
   a.x = *x; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.past_rows = pk ? past_rows : 0;
   a.qscale = scale * kLog2e;
   long rows = (long)x->T * Hq;
   long blocks = (rows + kWarps - 1) / kWarps;
@@ -135,12 +141,12 @@ int launch(const void *q, const void *k, const void *v, const void *pk, const vo
 }  // namespace
 
 int fork_attn_portable(const void *q, const void *k, const void *v, const void *pk,
-                       const void *pv, const flide_tree_index *x, int Hq, int Hkv, int d,
-                       int dtype, float scale, void *out, cudaStream_t s) {
+                       const void *pv, int past_rows, const flide_tree_index *x, int Hq,
+                       int Hkv, int d, int dtype, float scale, void *out, cudaStream_t s) {
   if (d <= 0 || d % 32 != 0 || d > 256) return FLIDE_ERR_SHAPE;
-  if (dtype == FLIDE_F32) return launch<float>(q, k, v, pk, pv, x, Hq, Hkv, d, scale, out, s);
+  if (dtype == FLIDE_F32) return launch<float>(q, k, v, pk, pv, past_rows, x, Hq, Hkv, d, scale, out, s);
   if (dtype == FLIDE_BF16)
-    return launch<__nv_bfloat16>(q, k, v, pk, pv, x, Hq, Hkv, d, scale, out, s);
+    return launch<__nv_bfloat16>(q, k, v, pk, pv, past_rows, x, Hq, Hkv, d, scale, out, s);
   return FLIDE_ERR_SHAPE;
 }
 

@@ -62,8 +62,8 @@
 
 namespace flide {
 int fork_attn_portable(const void *q, const void *k, const void *v, const void *pk,
-                       const void *pv, const flide_tree_index *x, int Hq, int Hkv, int d,
-                       int dtype, float scale, void *out, cudaStream_t s);
+                       const void *pv, int past_rows, const flide_tree_index *x, int Hq,
+                       int Hkv, int d, int dtype, float scale, void *out, cudaStream_t s);
 namespace {
 
 using namespace sm100;
@@ -125,6 +125,7 @@ struct TcParams {
   const int32_t *block_table, *req_slot;
   int max_blocks, block_rows, n_blocks, n_slots;
   int Hq, Hkv, G, mtok, has_past;  // mtok = tokens per 128-row half
+  int past_rows;                   // rows of the packed past buffers (unpaged)
   float qk_log2;                   // scale * log2(e)
 };
 
@@ -200,6 +201,15 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
     if (!p.has_past) {
       if (lane == 0) {
         set_status(x.status, FLIDE_ERR_SHAPE);
+        ms.valid = 0;
+      }
+      return;
+    }
+    // a packed past shorter than the tree's past rows: the tensor map would
+    // return zeros past its end, so refuse instead of attending to them
+    if (!p.block_table && (p0 < 0 || (long)p0 + plen > p.past_rows)) {
+      if (lane == 0) {
+        set_status(x.status, FLIDE_ERR_CAPACITY);
         ms.valid = 0;
       }
       return;
@@ -695,6 +705,7 @@ int fork_attn_tc(const void *q, const void *k, const void *v, const void *pk, co
   prm.G = G;
   prm.mtok = mtok;
   prm.has_past = has_past ? 1 : 0;
+  prm.past_rows = has_past ? past_rows : 0;
   prm.qk_log2 = scale * kLog2e;
   const long grid = (long)Hkv * ((x->T + 2 * mtok - 1) / (2 * mtok) + 2L * x->R);
   if (grid <= 0) return FLIDE_OK;
@@ -765,6 +776,6 @@ extern "C" int flide_fork_attn_noalloc(const void *q, const void *k, const void 
                         out, (cudaStream_t)stream, nullptr);
   }
   // the CUDA-core kernel keeps no per-call table
-  return fork_attn_portable(q, k, v, past_k, past_v, idx, Hq, Hkv, d, dtype, scale, out,
-                            (cudaStream_t)stream);
+  return fork_attn_portable(q, k, v, past_k, past_v, past_rows, idx, Hq, Hkv, d, dtype, scale,
+                            out, (cudaStream_t)stream);
 }

@@ -133,9 +133,53 @@ int plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *par
   return FLIDE_OK;
 }
 
+// Slots flide_tree_build assigns to the whole batch: every non-empty
+// request's root, plus the widest odd and even depth's inner nodes.
+int tree_state_slots(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
+                     int32_t *slots) {
+  if (R < 0 || !req_node_ptr || !slots) return FLIDE_ERR_SHAPE;
+  if (req_node_ptr[0] != 0) return FLIDE_ERR_INVALID;
+  for (int r = 0; r < R; ++r)
+    if (req_node_ptr[r + 1] < req_node_ptr[r]) return FLIDE_ERR_INVALID;
+  const int N = req_node_ptr[R];
+  if (N > 0 && !parent) return FLIDE_ERR_SHAPE;
+  std::vector<int> depth(N, 0), has_child(N, 0), inner_at_depth;
+  int roots = 0;
+  for (int r = 0; r < R; ++r) {
+    const int n0 = req_node_ptr[r], n1 = req_node_ptr[r + 1];
+    if (n1 > n0) ++roots;
+    for (int n = n0; n < n1; ++n) {
+      const int p = parent[n];
+      if (n == n0) {
+        if (p != -1) return FLIDE_ERR_INVALID;
+        continue;
+      }
+      if (p < 0 || n0 + p >= n) return FLIDE_ERR_INVALID;
+      depth[n] = depth[n0 + p] + 1;
+      has_child[n0 + p] = 1;
+    }
+  }
+  for (int n = 0; n < N; ++n)
+    if (has_child[n] && depth[n] >= 1) {
+      if ((int)inner_at_depth.size() <= depth[n]) inner_at_depth.resize(depth[n] + 1, 0);
+      ++inner_at_depth[depth[n]];
+    }
+  *slots = batch_slots(roots, inner_at_depth);
+  return FLIDE_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int flide_tree_state_slots(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
+                           int32_t *slots) {
+  try {  // no exception may cross the C ABI: out of host memory reads as capacity
+    return tree_state_slots(R, req_node_ptr, parent, slots);
+  } catch (...) {
+    return FLIDE_ERR_CAPACITY;
+  }
+}
 
 int flide_plan_state_groups(int32_t R, const int32_t *req_node_ptr, const int32_t *parent,
                             int32_t max_slots, int32_t *node_group, int32_t *n_groups) {

@@ -48,6 +48,20 @@ __device__ __forceinline__ int upper_bound(const int32_t *a, int n, int key) {
   return lo;
 }
 
+// Sum of one 64-bit value per thread across the block (blockDim.x a multiple
+// of 32, <= 1024); `scratch` holds >= 32 entries.
+__device__ long long block_sum_ll(long long v, long long *scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  long long tot = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += scratch[w];
+  __syncthreads();
+  return tot;
+}
+
 __global__ void __launch_bounds__(kNodeThreads)
 tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
   // capacities checked are the descriptor's (never above the index's)
@@ -90,9 +104,24 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
     return;
   }
 
+  // Totals in 64 bits first: the prefix sums below are int32 (the kernels'
+  // index type), so tokens beyond the capacity, or past rows plus tokens
+  // beyond 2^31 - 1 (positions, context lengths and checkpoint rows add
+  // them), are refused before any sum can wrap.
+  {
+    __shared__ long long sum_scratch[32];
+    long long ts = 0, ps = 0;
+    for (int n = tid; n < N; n += blockDim.x) ts += d.seg_len[n];
+    for (int r = tid; r < R; r += blockDim.x) ps += d.past_len[r];
+    ts = block_sum_ll(ts, sum_scratch);
+    ps = block_sum_ll(ps, sum_scratch);
+    if (ts > d.T || ts + ps > 0x7fffffffLL) {
+      if (tid == 0) set_status(x.status, FLIDE_ERR_CAPACITY);
+      return;
+    }
+  }
   const int T = block_scan_array(N, [&](int i) { return (int)d.seg_len[i]; }, x.node_start, scratch);
   const int P = block_scan_array(R, [&](int i) { return (int)d.past_len[i]; }, x.past_start, scratch);
-  if (tid == 0 && T > d.T) s_err = FLIDE_ERR_CAPACITY;
 
   // depth by walking parents (parent < self, so the walk ends)
   for (int n = tid; n < N; n += blockDim.x) {

@@ -35,7 +35,7 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
            "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_fork_attn_paged",
            "flide_plan_state_groups", "flide_copy_rows", "flide_fork_gdn_fp8", "flide_pool_append_batch",
-           "flide_strerror"]
+           "flide_tree_state_slots", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -126,6 +126,8 @@ def _lib():
         lib.flide_fork_attn_paged.restype = ctypes.c_int
         lib.flide_plan_state_groups.argtypes = [I32, P, P, I32, P, P]
         lib.flide_plan_state_groups.restype = ctypes.c_int
+        lib.flide_tree_state_slots.argtypes = [I32, P, P, P]
+        lib.flide_tree_state_slots.restype = ctypes.c_int
         lib.flide_copy_rows.argtypes = [P, P, P, P, I32, ctypes.c_int64, P]
         lib.flide_copy_rows.restype = ctypes.c_int
         lib.flide_fork_gdn_fp8.argtypes = [P, P, P, P, P, P, P, P, I32, I32, I32, P, P, I32, P]
@@ -577,25 +579,13 @@ def option_probs(index: TreeIndex, logp, path_logp=None, prob=None, stream=None)
 
 
 def state_slots(tree) -> int:
-    """Node-state slots that flide_tree_build assigns to a tree (counts["SLOTS"]):
-    one per request root, plus the largest number of inner nodes (nodes with
-    children) at any odd depth and at any even depth >= 2 -- inner nodes of
-    depth L share their region with depth L+2, which is written only after
-    depth L+1 has read them."""
+    """Node-state slots that flide_tree_build assigns to a tree (counts["SLOTS"]),
+    from the library's host query flide_tree_state_slots."""
     rp, parent, _seg, _past = tree.arrays()
-    R = len(rp) - 1
-    roots = int(sum(1 for r in range(R) if rp[r + 1] > rp[r]))
-    depth, inner = {}, set()
-    for r in range(R):
-        for n in range(rp[r], rp[r + 1]):
-            p = int(parent[n])
-            depth[n] = 0 if p < 0 else depth[rp[r] + p] + 1
-            if p >= 0:
-                inner.add(int(rp[r] + p))
-    per = {}
-    for n in inner:
-        if depth[n] >= 1:
-            per[depth[n]] = per.get(depth[n], 0) + 1
-    odd = max([c for d, c in per.items() if d % 2 == 1], default=0)
-    even = max([c for d, c in per.items() if d % 2 == 0], default=0)
-    return roots + odd + even
+    rp32 = np.ascontiguousarray(rp, np.int32)
+    pa32 = np.ascontiguousarray(parent, np.int32)
+    slots = ctypes.c_int32(0)
+    _check(_lib().flide_tree_state_slots(len(rp32) - 1, rp32.ctypes.data_as(ctypes.c_void_p),
+                                         pa32.ctypes.data_as(ctypes.c_void_p), ctypes.byref(slots)),
+           "flide_tree_state_slots")
+    return int(slots.value)
