@@ -432,6 +432,14 @@ def measure_workload(name, rank, steps, device, pg, local_rank, peak_tflops, hbm
     for _ in range(3):
         st.run()
     torch.cuda.synchronize()
+    # at least ~0.4 s of timed steps, so the clock sampler sees the load
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    st.run()
+    t1.record()
+    torch.cuda.synchronize()
+    steps = max(steps, min(2000, int(math.ceil(400.0 / max(t0.elapsed_time(t1), 1e-3)))))
+    steps = int(max_over_ranks(float(steps), pg, device))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     if pg is not None:
         pg.barrier()
@@ -490,7 +498,8 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the short timings of the other bf16 workloads")
     ap.add_argument("--workload-steps", type=int, default=10,
-                    help="timed steps per extra workload (after 3 warm-up steps)")
+                    help="least timed steps per extra workload (after 3 warm-up steps; more when a "
+                         "step is short, for about 0.4 s under load)")
     ap.add_argument("--vocab", type=int, default=8192, help="LM-head vocabulary of the decision leg")
     ap.add_argument("--cpu-rows", type=int, default=6000)
     ap.add_argument("--cpu-pairs", type=int, default=16)

@@ -57,6 +57,8 @@ extern "C" {
 #define FLIDE_ERR_CAPACITY 3 /* tree or data larger than the capacities given      */
 #define FLIDE_ERR_CUDA 4     /* a CUDA runtime call or kernel launch failed        */
 #define FLIDE_ERR_TIMEOUT 5  /* a bounded device-side wait expired                 */
+#define FLIDE_ERR_BOUNDS 6   /* bounds-checked build only: a data-dependent index left
+                                its array; the access was skipped (see flide_debug_bounds) */
 
 /* ---- element types ----------------------------------------------------- */
 #define FLIDE_F32 0
@@ -79,6 +81,8 @@ typedef void *flide_stream; /* cudaStream_t */
 #define FLIDE_CNT_BRANCH_TOK 5 /* tokens of non-root nodes                     */
 #define FLIDE_CNT_ROOT_TOK 6   /* tokens of root nodes                         */
 #define FLIDE_CNT_CKPT_ROWS 7  /* sum over requests of past_len + root seg_len */
+#define FLIDE_CNT_CHECK_SITE 12  /* first failed device check: its site number ...   */
+#define FLIDE_CNT_CHECK_VALUE 13 /* ... and the offending value (0 if none failed)   */
 
 /*
  * Tree descriptor: the request trees of one batch (kongchang.com,
@@ -537,6 +541,18 @@ int flide_copy_rows(void *dst, const void *src, const int32_t *dst_idx, const in
  * range. */
 int flide_selftest_wait_timeout(int32_t *status, int32_t timeout_us, int32_t arrive,
                                 flide_stream stream);
+
+/* Which build of the library is loaded: 1 for the bounds-checked debug build
+ * (libflide_dbg.so, compiled with FLIDE_DEBUG_BOUNDS), 0 for the release build.
+ * In the debug build every kernel checks the indices it takes from device data
+ * (tree arrays, work tables, block tables, state slots, token rows, TMA
+ * coordinates) against the array they index; a failed check skips the access
+ * (a read takes entry 0 instead, a write is dropped, a tile load is moved to
+ * row 0), records the check's site and value in counts[FLIDE_CNT_CHECK_SITE]
+ * and counts[FLIDE_CNT_CHECK_VALUE] (first failure wins) and writes
+ * FLIDE_ERR_BOUNDS to the status word -- never a trap or assert.  Both builds
+ * compute the same results on valid input.  Host only, no device access. */
+int32_t flide_debug_bounds(void);
 
 /* Static message for a status code ("unknown status" for any other value);
  * never NULL, owned by the library. */

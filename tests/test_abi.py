@@ -65,5 +65,7 @@ def test_host_only_entry_points():
     assert ptrs[-1] < base + n
     assert lib.flide_tree_index_init(ctypes.byref(idx), ctypes.c_void_p(base), n - 1, 4, 30, 1000, 3) == flide.ERR_CAPACITY
     assert lib.flide_tree_index_init(ctypes.byref(idx), ctypes.c_void_p(base + 4), n, 4, 30, 1000, 3) == flide.ERR_SHAPE
-    for code in range(6):
-        assert lib.flide_strerror(code)
+    for code in range(7):
+        assert lib.flide_strerror(code) and lib.flide_strerror(code) != b"unknown status"
+    assert lib.flide_strerror(7) == b"unknown status"
+    assert lib.flide_debug_bounds() == 0  # the release build

@@ -210,7 +210,7 @@ def test_fullsize_fork_attn_fp8_sampled(name):
     a = inputs.fp8_attn_inputs(tree, spec["Hq"], spec["Hkv"], spec["d"], rng)
     _, idx = build(tree)
     got, scale = _run_fp8(tree, a, idx)
-    rows = _rows(tree, spec["Hq"], 1500, np.random.default_rng(1))
+    rows = _rows(tree, spec["Hq"], spec["Hkv"], 1500, np.random.default_rng(1))
     want, tol = _oracle_and_bound(tree, a, scale, rows)
     _assert_within(got[rows[:, 0], rows[:, 1]], want, tol)
 

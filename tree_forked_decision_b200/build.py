@@ -1,9 +1,13 @@
 """Builds libflide.so in-tree with nvcc for sm_100a.
 
-    python -m tree_forked_decision_b200.build [--force]
+    python -m tree_forked_decision_b200.build [--force] [--debug-bounds]
 
 Each .cu under csrc/ is compiled separately (in parallel) and linked into
 tree_forked_decision_b200/libflide.so with the CUDA runtime linked statically.
+With --debug-bounds (build(debug_bounds=True)) the same sources are compiled
+with FLIDE_DEBUG_BOUNDS into libflide_dbg.so: every kernel then checks the
+indices it reads from device data and reports FLIDE_ERR_BOUNDS instead of
+making the access (the binding loads it when FLIDE_DEBUG_BOUNDS=1 is set).
 """
 from __future__ import annotations
 
@@ -20,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libflide.so")
+LIB_DBG = os.path.join(PKG, "libflide_dbg.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -44,22 +49,25 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
+    out_dir = os.path.join(BUILD, "dbg") if debug_bounds else BUILD
+    lib_path = LIB_DBG if debug_bounds else LIB
+    extra = ["-DFLIDE_DEBUG_BOUNDS"] if debug_bounds else []
+    os.makedirs(out_dir, exist_ok=True)
     nvcc = _nvcc()
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     objs = []
     jobs = []
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
             jobs.append((src, obj))
 
     def compile_one(job):
         src, obj = job
-        cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+        cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{res.stderr}")
@@ -69,15 +77,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
         for src, log in ex.map(compile_one, jobs):
             if verbose:
                 print(f"== {os.path.basename(src)}\n{log}")
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib_path, objs):
+        tmp = lib_path + f".tmp{os.getpid()}"
         cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                "-cudart", "static", "-o", tmp, *objs]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                debug_bounds="--debug-bounds" in sys.argv))

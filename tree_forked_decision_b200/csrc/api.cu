@@ -216,6 +216,8 @@ int flide_state_resume(int32_t R, const int32_t *src_req, int32_t src_R,
                       (cudaStream_t)stream);
 }
 
+int32_t flide_debug_bounds(void) { return kBoundsChecks ? 1 : 0; }
+
 const char *flide_strerror(int32_t code) {
   switch (code) {
     case FLIDE_OK: return "ok";
@@ -224,6 +226,7 @@ const char *flide_strerror(int32_t code) {
     case FLIDE_ERR_CAPACITY: return "tree or data exceeds the given capacities";
     case FLIDE_ERR_CUDA: return "CUDA call failed";
     case FLIDE_ERR_TIMEOUT: return "bounded device wait expired";
+    case FLIDE_ERR_BOUNDS: return "device index out of bounds (bounds-checked build)";
     default: return "unknown status";
   }
 }

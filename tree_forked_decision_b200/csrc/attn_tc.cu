@@ -174,6 +174,14 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
     return;
   }
   const int r = upper_bound_dev(x.work, R + 1, item) - 1;
+  const int Nact = x.counts[FLIDE_CNT_N], Tact = x.counts[FLIDE_CNT_T];
+  // debug build: the request, its root and its node range index the tree arrays
+  if (!in_bounds(x.status, x.counts, r, R, 201) ||
+      !in_bounds(x.status, x.counts, x.req_node[r], Nact, 202) ||
+      !in_bounds(x.status, x.counts, x.req_node[r + 1], Nact + 1, 203)) {
+    if (lane == 0) ms.valid = 0;
+    return;
+  }
   const int local = item - x.work[r];
   const int root = x.req_node[r];
   const int root_start = x.node_start[root];
@@ -232,9 +240,11 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
     for (int lvl = 1; lvl <= kMaxLevels; ++lvl) {
       int mn = INT_MAX, mx = -1;
       for (int i = lane; i < ntok; i += 32) {
-        const int n = x.token_node[t0 + i];
+        const int n = (int)checked(x.status, x.counts, x.token_node[checked(x.status, x.counts, t0 + i, Tact, 204)],
+                                   Nact, 205);
         if (x.depth[n] >= lvl) {
-          const int a = x.anc_node[x.anc_ptr[n] + lvl];
+          const int a = x.anc_node[checked(x.status, x.counts, (long long)x.anc_ptr[n] + lvl,
+                                           (long long)x.N * (x.max_depth + 1), 206)];
           mn = min(mn, a);
           mx = max(mx, a);
         }
@@ -242,11 +252,28 @@ __device__ void decode_item(const TcParams &p, Misc &ms, int lane) {
       mn = __reduce_min_sync(0xffffffffu, mn);
       mx = __reduce_max_sync(0xffffffffu, mx);
       if (mx < 0) break;
+      if (!in_bounds(x.status, x.counts, mn, Nact, 207) || !in_bounds(x.status, x.counts, mx, Nact, 207)) {
+        if (lane == 0) ms.valid = 0;
+        return;
+      }
       const int s0 = x.node_start[mn];
       sp[ns++] = Span{SRC_STREAM, s0, x.node_start[mx + 1] - s0, KIND_TREE, lvl, 0};
     }
   } else {
     sp[ns++] = Span{SRC_STREAM, root_start, t0 + ntok - root_start, KIND_CAUSAL, 0, 0};
+  }
+  // debug build: every stream span lies inside the stream, the tile's tokens too
+  for (int s = 0; s < ns; ++s)
+    if (sp[s].src == SRC_STREAM &&
+        (!in_bounds(x.status, x.counts, sp[s].start, Tact + 1, 208) ||
+         !in_bounds(x.status, x.counts, (long long)sp[s].start + sp[s].len, Tact + 1, 208))) {
+      if (lane == 0) ms.valid = 0;
+      return;
+    }
+  if (!in_bounds(x.status, x.counts, t0, Tact, 209) ||
+      !in_bounds(x.status, x.counts, (long long)t0 + ntok, Tact + 1, 209)) {
+    if (lane == 0) ms.valid = 0;
+    return;
   }
   int tiles = 0;
   for (int s = 0; s < ns; ++s) {
@@ -331,7 +358,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           int row = sp.start + off;
           if (sp.src == SRC_PAST && p.block_table) {
             // a key tile lies inside one block (block_rows % BN == 0)
-            int b = p.block_table[(size_t)ms.slot * p.max_blocks + off / p.block_rows];
+            int b = p.block_table[checked(x.status, x.counts,
+                                          (long long)ms.slot * p.max_blocks + off / p.block_rows,
+                                          (long long)p.n_slots * p.max_blocks, 210)];
             if (b < 0 || b >= p.n_blocks) {
               set_status(x.status, FLIDE_ERR_INVALID);  // no block: read block 0, flag the call
               b = 0;

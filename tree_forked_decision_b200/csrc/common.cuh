@@ -28,6 +28,31 @@ __device__ __forceinline__ bool failed(const int32_t *status) {
   return *(volatile const int32_t *)status != 0;
 }
 
+#ifdef FLIDE_DEBUG_BOUNDS
+constexpr bool kBoundsChecks = true;
+#else
+constexpr bool kBoundsChecks = false;
+#endif
+
+// Bounds check of an index taken from device data, compiled in only by the
+// debug build (FLIDE_DEBUG_BOUNDS).  Returns whether 0 <= i < n; on a failure
+// it records the site and the value in the index's check slots (first failure
+// wins) and FLIDE_ERR_BOUNDS in the status word, so the caller can skip the
+// access.  The release build folds every call to `true`.
+__device__ __forceinline__ bool in_bounds(int32_t *status, int32_t *counts, long long i,
+                                          long long n, int site) {
+  if (!kBoundsChecks || (i >= 0 && i < n)) return true;
+  if (atomicCAS(&counts[FLIDE_CNT_CHECK_SITE], 0, site) == 0)
+    counts[FLIDE_CNT_CHECK_VALUE] = (int32_t)i;
+  set_status(status, FLIDE_ERR_BOUNDS);
+  return false;
+}
+// i if it passes the check, else 0 (for reads that must still happen)
+__device__ __forceinline__ long long checked(int32_t *status, int32_t *counts, long long i,
+                                             long long n, int site) {
+  return in_bounds(status, counts, i, n, site) ? i : 0;
+}
+
 template <typename T>
 __device__ __forceinline__ float load_f(const T *p);
 template <>

@@ -186,11 +186,11 @@ __global__ void gdn_groups_kernel(flide_tree_index x, int level, int goff) {
   }
 }
 
-// Self-check: records the first failed bounds check (site, value) in the
-// index's spare count slots 12-13 and the status word; the caller skips the
-// access.
+// Self-check (both builds): records the first failed check of a work item
+// (site, value) in the index's check slots and FLIDE_ERR_INVALID in the status
+// word; the caller skips the item.
 __device__ __forceinline__ void check_fail(const flide_tree_index &x, int site, long val) {
-  if (atomicCAS(&x.counts[12], 0, site) == 0) x.counts[13] = (int)val;
+  if (atomicCAS(&x.counts[FLIDE_CNT_CHECK_SITE], 0, site) == 0) x.counts[FLIDE_CNT_CHECK_VALUE] = (int)val;
   set_status(x.status, FLIDE_ERR_INVALID);
 }
 
@@ -823,6 +823,813 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   }
 }
 
+// ---- warp-specialised fork scan ---------------------------------------------
+//
+// The same chunked form, with the chunk's work split by what it depends on.
+// Everything but the state products -- the segmented gate scan, [Q;K][Q;K]^T,
+// the decay masks, T = (I + A)^-1, W, U and the bf16 operand tiles -- depends
+// only on the chunk's own inputs, so a "prep" warpgroup computes it for chunk
+// c+1 while a "chain" warpgroup runs chunk c's state products:
+//   X = [U; 0] + [-W; diag(gamma) Q] S0^T       (rows 0-63: Delta, 64-127: gamma Q S0^T)
+//   X[64:] += (M o QK^T) Delta                   (the chunk's outputs)
+//   S = gamma_last S0 + Delta'^T K               (Delta' = Delta gamma_last / gamma)
+// With gamma folded into Q's rows the output needs no second accumulator; the
+// extra rounding is one bf16 rounding of gamma_i q_i, like the bf16 copy of S0.
+// Roles (384 threads): warps 0-3 chain (TMEM lanes 0-127), 4-7 prep, 8 producer
+// (items, per-token scalars, TMA), 10-11 epilogue (output rows, TMEM lanes
+// 64-127); warp 9 idles.  The producer runs ahead through a ring of four chunk
+// jobs, so the pipeline flows across items: a new item's first chunk starts
+// from its parent's state (global) while the previous item drains.  Every
+// handshake is an mbarrier whose next phase can only complete after its waiter
+// has consumed the current one, and every wait is bounded.  One thread of a
+// role polls a barrier while the rest of the role parks on a named barrier.  The chain's tiles
+// are single-buffered: the prep writes [-W; gamma Q] for chunk c+1 once chunk
+// c's first product has read them, and copies K once c's update has.
+namespace ws {
+
+constexpr int kThreads = 384;
+constexpr int kPrepWarp0 = 4, kProducerWarp = 8, kEpiWarp0 = 10;
+constexpr int BAR_PREP = 1, BAR_CHAIN = 2, BAR_EPI = 3;  // named barriers
+
+// shared-memory map, bytes from a 1024-aligned base
+constexpr int KQ = 0;          // stage s at +32768 s; dk slab b at +16384 b: Q rows at +0, K rows at +8192
+constexpr int V = 65536;       // dv slab b at +8192 b (64 token rows)
+constexpr int MQK = 81920;     // stage s at +8192 s: rows 64-127 of a [junk; M o QK^T] A tile
+constexpr int CA = 98304;      // [-W; gamma Q] A tile, dk slab b at +16384 b
+constexpr int CK = 131072;     // K rows for the state update (MN-major B), dk slab b at +8192 b
+constexpr int SD = 147456;     // bf16 S0 (dk slab b at +16384 b); then Delta (+0) and Delta' (+16384)
+constexpr int TT = 180224;     // T' (+0), T'' (+8192), zeros (+16384); solve scratch during the solve
+constexpr int PM = 204800;     // fp32 [64][65]: T below the diagonal, A^T above it
+constexpr int P_LD = 65;
+constexpr int JOB = PM + C * P_LD * 4;  // 4 chunk jobs
+constexpr int JOB_BYTES = 1600;
+constexpr int BARS = JOB + 4 * JOB_BYTES;
+enum {
+  KQ_FULL = 0, KQ_EMPTY = 2, V_FULL = 4, V_EMPTY = 5, JOB_FULL = 6, JOB_FREE = 10, GRAM = 14,
+  WU = 15, READY = 16, CA_FREE = 17, XDONE = 18, SO = 19, XFREE = 21, DRAIN_P = 23,
+  DRAIN_C = 24, CK_FREE = 25, NBARS = 26
+};
+constexpr int MISC = BARS + 8 * NBARS;  // TMEM address, abort flag
+constexpr int SMEM_BYTES = MISC + 16 + 1024;
+static_assert(JOB % 16 == 0 && BARS % 8 == 0, "job slots and barriers must be aligned");
+static_assert(SMEM_BYTES <= 232448, "shared memory over the 227 KB limit");
+
+// TMEM columns
+constexpr uint32_t T_S = 0, T_X0 = 128, T_X1 = 256, T_G = 384;
+
+// One chunk of one (item, head), written by the producer: header, beta, the
+// segmented log2 decay G2, gamma = 2^G2, the separable decay factors
+// f_j = 2^(gref - G2_j), the state-update scales gamma_last / gamma_j and each
+// token's segment start; read by the prep, the chain and the epilogue.
+struct Job {
+  int stop, cbeg, n, h, first, update, save, sep;
+  const float *src;  // first chunk: start state [dv][dk], nullptr = zero
+  float *dst;        // save: end state [dv][dk]
+  float gam_last, gref, pad0, pad1;
+  float beta[C], g2[C], gam[C], f[C], dsc[C];
+  int lo[C];  // first token of the token's segment (C for tokens past the chunk)
+};
+static_assert(sizeof(Job) <= JOB_BYTES, "job slot too small");
+
+__device__ __forceinline__ void role_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// every thread of the role gets the AND of the role's predicates
+__device__ __forceinline__ bool role_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// fp32 tile entry T(r, c) of the solve area: below the diagonal the solved
+// value, 1 on it, 0 above (where A^T is kept)
+__device__ __forceinline__ float t_at(const float *Pm, int r, int c) {
+  return r > c ? Pm[r * P_LD + c] : (r == c ? 1.f : 0.f);
+}
+// A(r, c) for r > c, kept transposed above the diagonal
+__device__ __forceinline__ float a_at(const float *Pm, int r, int c) { return Pm[c * P_LD + r]; }
+
+// acc (16 x 8) += X (16 x 16) Y (16 x 8) with tf32 inputs (m16n8k8, two K
+// steps); X and Y given as element functions
+template <typename FX, typename FY>
+__device__ __forceinline__ void mma16x8(float (&acc)[4], FX X, FY Y, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kk = 0; kk < 16; kk += 8) {
+    mma_tf32_16x8x8(acc, to_tf32(X(g, kk + t)), to_tf32(X(g + 8, kk + t)), to_tf32(X(g, kk + t + 4)),
+                    to_tf32(X(g + 8, kk + t + 4)), to_tf32(Y(kk + t, g)), to_tf32(Y(kk + t + 4, g)));
+  }
+}
+
+}  // namespace ws
+
+template <bool F8>
+__global__ void __launch_bounds__(ws::kThreads, 1)
+gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const GdnTcParams p) {
+  using namespace ws;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-aligned base by pointer arithmetic on the shared array, so the
+  // compiler keeps the shared address space (shared, not generic, accesses)
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const flide_tree_index &x = p.x;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + MISC);
+  int *abort_flag = reinterpret_cast<int *>(smem + MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return sb + BARS + 8 * i; };
+  auto job = [&](int j) -> Job * { return reinterpret_cast<Job *>(smem + JOB + j * JOB_BYTES); };
+  const float dsq = F8 ? p.descale[0] : 1.f, dsk = F8 ? p.descale[1] : 1.f,
+              dsv = F8 ? p.descale[2] : 1.f;
+
+  if (tid == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i >= JOB_FREE && i < JOB_FREE + 4 ? 2 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // the zero rows of the [T''; 0] tile
+  for (int i = tid; i < 8192 / 16; i += ws::kThreads)
+    reinterpret_cast<uint4 *>(smem + TT + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (warp == 0) {
+    tmem_alloc(sb + MISC, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int *vabort = abort_flag;
+  const int Tact = x.counts[FLIDE_CNT_T];
+
+  if (warp == kProducerWarp) {
+    // ---------------- producer: items -> chunk jobs, per-token scalars, TMA
+    const int n_groups = failed(x.status) ? 0 : *groups_n(x, p.goff);
+    const int L0 = x.level_ptr[p.level];
+    const long long items = (long long)n_groups * p.H;
+    const int Nact = x.counts[FLIDE_CNT_N];
+    uint32_t seq = 0;
+    int last_kq[2] = {-1, -1}, last_v = -1;  // last issued load per buffer (drain)
+    bool ok = true;
+    auto wait_w = [&](uint32_t b, uint32_t parity) -> bool {  // lane 0 polls
+      bool r = true;
+      if (lane == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
+      return __shfl_sync(0xffffffffu, (int)r, 0) != 0;
+    };
+    // claims job slot `seq` (all lanes), false if the wait gave up
+    auto claim = [&](Job *&jb) -> bool {
+      if (!wait_w(bar(JOB_FREE + (seq & 3)), ((seq >> 2) & 1) ^ 1)) return false;
+      jb = job(seq & 3);
+      return true;
+    };
+    for (;;) {
+      unsigned long long it = 0;
+      if (lane == 0) it = (unsigned long long)atomicAdd(groups_next(x, p.goff), 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      bool stop = (long long)it >= items || *vabort;
+      int h = 0, tbeg = 0, tend = 0, n0 = 0, slot = -1, r = 0, cnt = 0;
+      const float *src = nullptr;
+      if (!stop) {
+        const int rk = (int)(it / p.H);
+        h = (int)(it % p.H);
+        const int grp = groups_order(x, p.goff)[rk];
+        int site = 0;
+        long val = 0;
+        int k0 = 0;
+        if (grp < 0 || grp >= n_groups) {
+          site = 6; val = grp;
+        } else {
+          k0 = groups_start(x, p.goff)[grp];
+          cnt = groups_count(x, p.goff)[grp];
+          if (k0 < 0 || cnt < 1 || L0 + k0 + cnt > Nact) { site = 1; val = k0 * 100000L + cnt; }
+        }
+        int n1 = 0;
+        if (!site) {
+          n0 = x.level_node[L0 + k0];
+          n1 = x.level_node[L0 + k0 + cnt - 1];
+          if (n0 < 0 || n1 < n0 || n1 >= Nact) { site = 2; val = n0 * 100000L + n1; }
+        }
+        if (!site) {
+          tbeg = x.node_start[n0];
+          tend = x.node_start[n1 + 1];
+          if (tbeg < 0 || tend < tbeg || tend > Tact) { site = 3; val = tend; }
+        }
+        if (!site) {
+          slot = x.state_slot[n0];
+          r = x.node_req[n0];
+          if (r < 0 || r >= x.R || (slot >= 0 && slot >= p.n_slots)) { site = 4; val = r * 100000L + slot; }
+        }
+        if (!site) {
+          if (p.level == 0) {
+            if (p.state_in) src = p.state_in + ((size_t)r * p.H + h) * D * D;
+          } else {
+            const int pa = x.anc_ptr[n0 + 1] - 2;
+            const int ps = (pa >= 0 && x.depth[n0] >= 1) ? x.state_slot[x.anc_node[pa]] : -1;
+            if (ps < 0 || ps >= p.n_slots) { site = 5; val = ps; }
+            else src = p.node_state + ((size_t)ps * p.H + h) * D * D;
+          }
+        }
+        if (site) {
+          if (lane == 0) check_fail(x, site, val);
+          stop = true;
+        }
+      }
+      if (stop) {
+        Job *jb;
+        if (!claim(jb)) { ok = false; break; }
+        if (lane == 0) jb->stop = 1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(JOB_FULL + (seq & 3)));
+        break;
+      }
+      const bool scan = cnt == 1;
+      float *dst = (scan && slot >= 0) ? p.node_state + ((size_t)slot * p.H + h) * D * D : nullptr;
+      const int nchunks = (tend - tbeg + C - 1) / C;
+      if (nchunks == 0) {
+        // a node without tokens (a root whose prefix is all past): its end
+        // state is its start state
+        if (dst) {
+          for (int i = lane; i < D * D / 4; i += 32)
+            reinterpret_cast<float4 *>(dst)[i] =
+                src ? reinterpret_cast<const float4 *>(src)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
+      }
+      for (int c = 0; c < nchunks; ++c, ++seq) {
+        Job *jb;
+        if (!claim(jb)) { ok = false; break; }
+        const int cbeg = tbeg + c * C;
+        const int n = min(C, tend - cbeg);
+        // K and Q into stage s first, so the copy overlaps the scalar work
+        const int s = seq & 1;
+        if (!wait_w(bar(KQ_EMPTY + s), ((seq >> 1) & 1) ^ 1)) { ok = false; break; }
+        if (lane == 0) {
+          const uint32_t kq = sb + KQ + s * 32768, fb = bar(KQ_FULL + s);
+          mbar_arrive_expect_tx(fb, 32768);
+          tma_load_3d(kq, &tm_q, fb, 0, h, cbeg);
+          tma_load_3d(kq + 16384, &tm_q, fb, 64, h, cbeg);
+          tma_load_3d(kq + 8192, &tm_k, fb, 0, h, cbeg);
+          tma_load_3d(kq + 16384 + 8192, &tm_k, fb, 64, h, cbeg);
+        }
+        last_kq[s] = (int)(seq >> 1);
+        if (lane == 0) {
+          jb->stop = 0;
+          jb->cbeg = cbeg;
+          jb->n = n;
+          jb->h = h;
+          jb->first = c == 0;
+          jb->update = scan && (c + 1 < nchunks || slot >= 0);
+          jb->save = scan && slot >= 0 && c + 1 == nchunks;
+          jb->src = src;
+          jb->dst = dst;
+        }
+        {
+          // per-token scalars, two consecutive tokens per lane, and the
+          // segmented inclusive scan of g (segments = nodes of a packed group)
+          const int t0 = 2 * lane, t1 = t0 + 1;
+          const bool v0 = t0 < n && cbeg + t0 < Tact, v1 = t1 < n && cbeg + t1 < Tact;
+          const size_t i0 = (size_t)(cbeg + t0) * p.H + h, i1 = i0 + p.H;
+          const float b0 = v0 ? p.beta[i0] : 0.f, b1 = v1 ? p.beta[i1] : 0.f;
+          const float a0 = v0 ? p.g[i0] : 0.f, a1 = v1 ? p.g[i1] : 0.f;
+          const int s0 = v0 ? x.token_node[cbeg + t0] - n0 : -1;
+          const int s1 = v1 ? x.token_node[cbeg + t1] - n0 : -1;
+          const int prev_s1 = __shfl_up_sync(0xffffffffu, s1, 1);
+          const bool cont0 = lane > 0 && prev_s1 == s0;  // token t0 continues token t0 - 1
+          float v = (s1 == s0) ? a0 + a1 : a1;
+          int f = (s1 != s0 || !cont0) ? 1 : 0;
+          // segment starts: the latest start at or before each token
+          const int st0 = cont0 ? -1 : t0, st1 = (s1 == s0) ? -1 : t1;
+          int m = max(st0, st1);
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float pv = __shfl_up_sync(0xffffffffu, v, o);
+            const int pf = __shfl_up_sync(0xffffffffu, f, o);
+            const int pm = __shfl_up_sync(0xffffffffu, m, o);
+            if (lane >= o) {
+              if (!f) v += pv;
+              f |= pf;
+              m = max(m, pm);
+            }
+          }
+          const float carry = __shfl_up_sync(0xffffffffu, v, 1);
+          const int mprev = __shfl_up_sync(0xffffffffu, m, 1);
+          const int lo0 = max(lane > 0 ? mprev : -1, st0), lo1 = max(lo0, st1);
+          const float G0 = a0 + (cont0 ? carry : 0.f);
+          const float g0 = G0 * 1.4426950408889634f;
+          const float g1 = ((s1 == s0) ? G0 + a1 : a1) * 1.4426950408889634f;
+          float mx = fmaxf(v0 ? g0 : -INFINITY, v1 ? g1 : -INFINITY);
+          float mn = fminf(v0 ? g0 : INFINITY, v1 ? g1 : INFINITY);
+          mx = warp_max(mx);
+          mn = -warp_max(-mn);
+          const bool sep = !(mx - mn > 100.f);  // also true when no token is valid
+          const float gref = (mx >= mn) ? 0.5f * (mx + mn) : 0.f;
+          const float glast = __shfl_sync(0xffffffffu, (n - 1) & 1 ? g1 : g0, (n - 1) >> 1);
+          jb->beta[t0] = b0;
+          jb->beta[t1] = b1;
+          jb->g2[t0] = g0;
+          jb->g2[t1] = g1;
+          jb->gam[t0] = ex2_approx(g0);
+          jb->gam[t1] = ex2_approx(g1);
+          jb->f[t0] = sep ? ex2_approx(gref - g0) : 0.f;
+          jb->f[t1] = sep ? ex2_approx(gref - g1) : 0.f;
+          jb->dsc[t0] = v0 ? ex2_approx(glast - g0) : 0.f;
+          jb->dsc[t1] = v1 ? ex2_approx(glast - g1) : 0.f;
+          jb->lo[t0] = v0 ? lo0 : C;
+          jb->lo[t1] = v1 ? lo1 : C;
+          if (lane == 0) {
+            jb->gam_last = ex2_approx(glast);
+            jb->gref = gref;
+            jb->sep = sep ? 1 : 0;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(JOB_FULL + (seq & 3)));
+        // V
+        if (!wait_w(bar(V_EMPTY), (seq & 1) ^ 1)) { ok = false; break; }
+        if (lane == 0) {
+          const uint32_t vb = sb + V, fb = bar(V_FULL);
+          mbar_arrive_expect_tx(fb, 16384);
+          tma_load_3d(vb, &tm_v, fb, 0, h, cbeg);
+          tma_load_3d(vb + 8192, &tm_v, fb, 64, h, cbeg);
+        }
+        last_v = (int)seq;
+      }
+      if (!ok) break;
+    }
+    // every issued load lands before the CTA can exit
+    if (lane == 0) {
+      for (int s = 0; s < 2; ++s)
+        if (last_kq[s] >= 0) mbar_wait(bar(KQ_FULL + s), last_kq[s] & 1, vabort, kTimeoutNs, false);
+      if (last_v >= 0) mbar_wait(bar(V_FULL), last_v & 1, vabort, kTimeoutNs, false);
+    }
+    __syncwarp();
+  } else if (warp >= kPrepWarp0 && warp < kPrepWarp0 + 4) {
+    // ---------------- prep: everything of a chunk that does not need the state
+    const int pt = tid - kPrepWarp0 * 32;
+    const uint32_t tlp = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    float *Pm = reinterpret_cast<float *>(smem + PM);
+    float *Xs = reinterpret_cast<float *>(smem + TT);  // 4 blocks of 16 x 17 during the solve
+    constexpr int XS_LD = 17;
+    bool issued = false;  // MMAs in flight (pt == 0), for the drain
+    auto wait_r = [&](uint32_t b, uint32_t parity) -> bool {  // one poller, the rest park
+      bool r = true;
+      if (pt == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
+      return role_and(BAR_PREP, 128, r);
+    };
+    for (uint32_t seq = 0;; ++seq) {
+      if (!wait_r(bar(JOB_FULL + (seq & 3)), (seq >> 2) & 1)) break;
+      Job *jb = job(seq & 3);
+      if (jb->stop) break;
+      const int n = jb->n, s = seq & 1;
+      const uint32_t kq = sb + KQ + s * 32768;
+      uint8_t *kqp = smem + KQ + s * 32768;
+      // -- 2. this chunk's Q and K; rows past the chunk's tokens zeroed (they
+      //       may hold another node's tokens or uninitialised memory)
+      if (!wait_r(bar(KQ_FULL + s), (seq >> 1) & 1)) break;
+      if (n < C) {
+        for (int e = pt; e < 4 * C * 8; e += 128) {  // (slab, Q|K, row, 16-byte chunk)
+          const int row = (e >> 3) & (C - 1);
+          if (row >= n)
+            *reinterpret_cast<uint4 *>(kqp + (e >> 10) * 16384 + ((e >> 9) & 1) * 8192 + row * 128 +
+                                       (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      role_sync(BAR_PREP, 128);
+      if (pt == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = sdesc_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_bf16(tmem + T_G, d, d, id, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(GRAM));
+        issued = true;
+      }
+      __syncwarp();
+      if (!wait_r(bar(GRAM), seq & 1)) break;
+      tc_fence_after();
+      // -- 3. decay masks from the Gram columns 64-127 (k_j): rows 0-63 are
+      //       q_i . k_j -> (M o QK^T) in bf16; rows 64-127 are k_i . k_j -> A
+      //       (fp32, kept transposed above the diagonal of the solve area)
+      {
+        const bool sep = jb->sep != 0;
+        const bool qrow = pt < C;
+        const int i = pt & (C - 1);
+        const float G2i = jb->g2[i];
+        const int lo = jb->lo[i], hi = qrow ? i : i - 1;  // visible j: lo <= j <= hi
+        const float sc = qrow ? dsq * dsk : jb->beta[i] * (dsk * dsk);
+        const float ei = sc * (sep ? ex2_approx(G2i - jb->gref) : 1.f);
+        uint32_t d[64];
+        tmem_ld64(tlp + T_G + 64, d);
+        uint8_t *mq = smem + MQK + s * 8192;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // 8 columns at a time: few live registers
+          const float4 fa = reinterpret_cast<const float4 *>(sep ? jb->f : jb->g2)[2 * q];
+          const float4 fb = reinterpret_cast<const float4 *>(sep ? jb->f : jb->g2)[2 * q + 1];
+          const float fj[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+          float e[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 8 * q + u;
+            const float ratio = sep ? ei * fj[u] : ei * ex2_approx(G2i - fj[u]);
+            e[u] = (j >= lo && j <= hi) ? ratio * __uint_as_float(d[j]) : 0.f;
+          }
+          if (qrow) {
+            st_chunk(mq, i, q, pack8(e));
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              if (8 * q + u < i) Pm[(8 * q + u) * P_LD + i] = e[u];
+          }
+        }
+      }
+      role_sync(BAR_PREP, 128);
+      // -- 4. T = (I + A)^-1: the four diagonal 16 x 16 blocks by substitution,
+      //       then the off-diagonal blocks by doubling: T_10, T_32 from
+      //       T_ii (-A_ij) T_jj, then the lower-left 32 x 32 block the same way
+      if (pt < C) {
+        const int r0 = 16 * (pt >> 4), cc = pt & 15;
+        float tcol[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int j = 0; j + 1 < i; j += 2) {
+            s0 = fmaf(a_at(Pm, r0 + i, r0 + j), tcol[j], s0);
+            s1 = fmaf(a_at(Pm, r0 + i, r0 + j + 1), tcol[j + 1], s1);
+          }
+          if (i & 1) s0 = fmaf(a_at(Pm, r0 + i, r0 + i - 1), tcol[i - 1], s0);
+          tcol[i] = (i == cc) ? 1.f : (i > cc ? -(s0 + s1) : 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i > cc) Pm[(r0 + i) * P_LD + r0 + cc] = tcol[i];
+      }
+      role_sync(BAR_PREP, 128);
+      {
+        // T_10 (warps 4, 5: column halves) and T_32 (warps 6, 7)
+        const int wq = warp - kPrepWarp0;
+        const int I = (wq >> 1) ? 3 : 1, J = I - 1, half = wq & 1;
+        const int rI = 16 * I, cJ = 16 * J, cn = cJ + 8 * half;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma16x8(acc, [&](int r, int k) { return a_at(Pm, rI + r, cJ + k); },
+                [&](int k, int c) { return t_at(Pm, cJ + k, cn + c); }, lane);
+        float *xs = Xs + wq * 16 * XS_LD;
+        const int g = lane >> 2, t = lane & 3;
+        xs[g * XS_LD + 2 * t] = acc[0];
+        xs[g * XS_LD + 2 * t + 1] = acc[1];
+        xs[(g + 8) * XS_LD + 2 * t] = acc[2];
+        xs[(g + 8) * XS_LD + 2 * t + 1] = acc[3];
+        __syncwarp();
+        float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+        mma16x8(acc2, [&](int r, int k) { return t_at(Pm, rI + r, rI + k); },
+                [&](int k, int c) { return xs[k * XS_LD + c]; }, lane);
+        Pm[(rI + g) * P_LD + cn + 2 * t] = -acc2[0];
+        Pm[(rI + g) * P_LD + cn + 2 * t + 1] = -acc2[1];
+        Pm[(rI + g + 8) * P_LD + cn + 2 * t] = -acc2[2];
+        Pm[(rI + g + 8) * P_LD + cn + 2 * t + 1] = -acc2[3];
+      }
+      role_sync(BAR_PREP, 128);
+      {
+        // lower-left 32 x 32: X_IJ = sum_{K=J..1} A_IK T_KJ, then
+        // T_IJ = -sum_{K=2..I} T_IK X_KJ; warp (I, J) = 4:(2,0) 5:(2,1) 6:(3,0) 7:(3,1)
+        const int wq = warp - kPrepWarp0;
+        const int I = 2 + (wq >> 1), J = wq & 1;
+        const int g = lane >> 2, t = lane & 3;
+        float *xs = Xs + wq * 16 * XS_LD;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int K = 0; K <= 1; ++K)
+            if (K >= J)
+              mma16x8(acc, [&](int r, int k) { return a_at(Pm, 16 * I + r, 16 * K + k); },
+                      [&](int k, int c) { return t_at(Pm, 16 * K + k, 16 * J + 8 * nt + c); }, lane);
+          xs[g * XS_LD + 8 * nt + 2 * t] = acc[0];
+          xs[g * XS_LD + 8 * nt + 2 * t + 1] = acc[1];
+          xs[(g + 8) * XS_LD + 8 * nt + 2 * t] = acc[2];
+          xs[(g + 8) * XS_LD + 8 * nt + 2 * t + 1] = acc[3];
+        }
+        role_sync(BAR_PREP, 128);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int K = 2; K <= 3; ++K) {
+            if (K > I) continue;
+            const float *xk = Xs + (2 * (K - 2) + J) * 16 * XS_LD;
+            mma16x8(acc, [&](int r, int k) { return t_at(Pm, 16 * I + r, 16 * K + k); },
+                    [&](int k, int c) { return xk[k * XS_LD + 8 * nt + c]; }, lane);
+          }
+          const int cn = 16 * J + 8 * nt;
+          Pm[(16 * I + g) * P_LD + cn + 2 * t] = -acc[0];
+          Pm[(16 * I + g) * P_LD + cn + 2 * t + 1] = -acc[1];
+          Pm[(16 * I + g + 8) * P_LD + cn + 2 * t] = -acc[2];
+          Pm[(16 * I + g + 8) * P_LD + cn + 2 * t + 1] = -acc[3];
+        }
+      }
+      role_sync(BAR_PREP, 128);
+      // -- 5. T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles
+      {
+        const int i = pt >> 1, half = pt & 1;
+        uint8_t *t1 = smem + TT, *t2 = smem + TT + 8192;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float f1[8], f2[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 32 * half + 8 * q + u;
+            const float tv = t_at(Pm, i, j), b = jb->beta[j];
+            f1[u] = tv * (b * jb->gam[j] * dsk);
+            f2[u] = tv * (b * dsv);
+          }
+          st_chunk(t1, i, 4 * half + q, pack8(f1));
+          st_chunk(t2, i, 4 * half + q, pack8(f2));
+        }
+      }
+      // -- 6. V (rows past the chunk zeroed), then W = T' K -> T_G and
+      //       U = [T''; 0] V -> X[s] once the epilogue of chunk seq-2 has read X[s]
+      if (!wait_r(bar(V_FULL), seq & 1)) break;
+      if (n < C) {
+        for (int e = pt; e < 2 * C * 8; e += 128) {
+          const int row = (e >> 3) & (C - 1);
+          if (row >= n)
+            *reinterpret_cast<uint4 *>(smem + V + (e >> 9) * 8192 + row * 128 + (e & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      if (!wait_r(bar(XFREE + s), ((seq >> 1) & 1) ^ 1)) break;
+      if (pt == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, true);
+        const uint32_t xs_t = tmem + (s ? T_X1 : T_X0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_bf16(tmem + T_G, sdesc_sw128(sb + TT + kk * 32, 16, 1024),
+                   sdesc_sw128(kq + 8192 + kk * 2048, 16384, 1024), id, kk > 0 ? 1u : 0u);
+          mma_bf16(xs_t, sdesc_sw128(sb + TT + 8192 + kk * 32, 16, 1024),
+                   sdesc_sw128(sb + V + kk * 2048, 8192, 1024), id, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(WU));
+      }
+      __syncwarp();
+      if (!wait_r(bar(WU), seq & 1)) break;
+      tc_fence_after();
+      if (pt == 0) mbar_arrive(bar(V_EMPTY));
+      // -- 7. the chain's tiles, each once chunk seq-1's chain has finished
+      //       with it: [-W; gamma Q] after its first product, K after the update
+      if (!wait_r(bar(CA_FREE), (seq & 1) ^ 1)) break;
+      if (pt < C) {
+        const int i = pt;  // W row = token (TMEM lanes 0-63)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          uint32_t w[64];
+          tmem_ld64(tlp + T_G + 64 * b, w);
+          uint8_t *dst = smem + CA + b * 16384;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(w[8 * q + u]);
+            st_chunk(dst, i, q, pack8(f));
+          }
+        }
+      } else {
+        const int i = pt - C;  // gamma_i q_i into tile rows 64-127 (same swizzle phase)
+        const float gq = jb->gam[i] * dsq;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int off = i * 128 + ((q ^ (i & 7)) << 4);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(kqp + b * 16384 + off);
+            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[u]));
+              f[2 * u] = v2.x * gq;
+              f[2 * u + 1] = v2.y * gq;
+            }
+            *reinterpret_cast<uint4 *>(smem + CA + b * 16384 + 8192 + off) = pack8(f);
+          }
+        }
+      }
+      if (!wait_r(bar(CK_FREE), (seq & 1) ^ 1)) break;
+      for (int e = pt; e < 2 * C * 8; e += 128) {  // K rows: same rows, same swizzle
+        const int b = e >> 9, rest = (e & 511) * 16;
+        *reinterpret_cast<uint4 *>(smem + CK + b * 8192 + rest) =
+            *reinterpret_cast<const uint4 *>(kqp + b * 16384 + 8192 + rest);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      role_sync(BAR_PREP, 128);
+      if (pt == 0) {
+        mbar_arrive(bar(READY));
+        mbar_arrive(bar(KQ_EMPTY + s));
+      }
+    }
+    if (pt == 0 && issued && *vabort) {  // MMAs still in flight after a timeout
+      mma_commit(bar(DRAIN_P));
+      mbar_wait(bar(DRAIN_P), 0, vabort, kTimeoutNs, false);
+    }
+  } else if (warp < 4) {
+    // ---------------- chain: the state products, chunk after chunk
+    const int row = tid;  // TMEM lane = state row (dv) / token row
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    bool issued = false;
+    auto wait_r = [&](uint32_t b, uint32_t parity) -> bool {  // one poller, the rest park
+      bool r = true;
+      if (tid == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
+      return role_and(BAR_CHAIN, 128, r);
+    };
+    for (uint32_t seq = 0;; ++seq) {
+      const int j = seq & 3;
+      if (!wait_r(bar(JOB_FULL + j), (seq >> 2) & 1)) break;
+      Job *jb = job(j);
+      if (jb->stop) break;
+      const int s = seq & 1;
+      const bool first = jb->first, update = jb->update, save = jb->save;
+      const float *src = jb->src;
+      float *dst = jb->dst;
+      if (!wait_r(bar(READY), seq & 1)) break;
+      const float gl = jb->gam_last;
+      const uint32_t xt = s ? T_X1 : T_X0;
+      // -- S0 as the bf16 B operand; S <- gamma_last S for the update
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        uint32_t v[64];
+        if (first) {
+#pragma unroll
+          for (int i = 0; i < 64; i += 4) {
+            const float4 f4 = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * D + 64 * b + i)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[i] = __float_as_uint(f4.x);
+            v[i + 1] = __float_as_uint(f4.y);
+            v[i + 2] = __float_as_uint(f4.z);
+            v[i + 3] = __float_as_uint(f4.w);
+          }
+        } else {
+          tmem_ld64(tl + T_S + 64 * b, v);
+        }
+        uint8_t *s0 = smem + SD + b * 16384;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(v[8 * q + u]);
+          st_chunk(s0, row, q, pack8(f));
+        }
+        if (update) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * gl);
+          tmem_st64(tl + T_S + 64 * b, v);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      role_sync(BAR_CHAIN, 128);
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16(tmem + xt, sdesc_sw128(sb + CA + o, 16, 1024), sdesc_sw128(sb + SD + o, 16, 1024),
+                   id, 1u);
+        }
+        mma_commit(bar(XDONE));
+        issued = true;
+      }
+      __syncwarp();
+      if (!wait_r(bar(XDONE), seq & 1)) break;
+      tc_fence_after();
+      if (tid == 0) mbar_arrive(bar(CA_FREE));
+      // -- Delta (token rows 0-63) as the MN-major B of (M o QK^T) Delta, and
+      //    Delta' = Delta gamma_last / gamma_j as the MN-major A of the update
+      if (row < C) {
+        const float dj = jb->dsc[row] * dsk;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          uint32_t v[64];
+          tmem_ld64(tl + xt + 64 * b, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float f[8], f2[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              f[u] = __uint_as_float(v[8 * q + u]);
+              f2[u] = f[u] * dj;
+            }
+            st_chunk(smem + SD + b * 8192, row, q, pack8(f));
+            if (update) st_chunk(smem + SD + 16384 + b * 8192, row, q, pack8(f2));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      role_sync(BAR_CHAIN, 128);
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t mq = sb + MQK + s * 8192 - 8192;  // [junk; M o QK^T]
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          if (update)
+            mma_bf16(tmem + T_S, sdesc_sw128(sb + SD + 16384 + kk * 2048, 8192, 1024),
+                     sdesc_sw128(sb + CK + kk * 2048, 8192, 1024),
+                     idesc_bf16_ex(128, 128, true, true, false), 1u);
+          mma_bf16(tmem + xt, sdesc_sw128(mq + kk * 32, 16, 1024),
+                   sdesc_sw128(sb + SD + kk * 2048, 8192, 1024), idesc_bf16(128, 128, true), 1u);
+        }
+        mma_commit(bar(SO + s));
+      }
+      __syncwarp();
+      if (!wait_r(bar(SO + s), (seq >> 1) & 1)) break;
+      tc_fence_after();
+      if (tid == 0) {
+        mbar_arrive(bar(CK_FREE));
+        mbar_arrive(bar(JOB_FREE + j));
+      }
+      if (save) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          uint32_t v[64];
+          tmem_ld64(tl + T_S + 64 * b, v);
+          float *d = dst + (size_t)row * D + 64 * b;
+#pragma unroll
+          for (int i = 0; i < 64; i += 4)
+            *reinterpret_cast<float4 *>(d + i) =
+                make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                            __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        }
+      }
+    }
+    if (tid == 0 && issued && *vabort) {
+      mma_commit(bar(DRAIN_C));
+      mbar_wait(bar(DRAIN_C), 0, vabort, kTimeoutNs, false);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------- epilogue: output rows (TMEM lanes 64-127 of X)
+    const int i = tid - kEpiWarp0 * 32;  // token of the chunk
+    const uint32_t tle = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    auto wait_r = [&](uint32_t b, uint32_t parity) -> bool {  // one poller, the rest park
+      bool r = true;
+      if (i == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
+      return role_and(BAR_EPI, 64, r);
+    };
+    for (uint32_t seq = 0;; ++seq) {
+      const int j = seq & 3;
+      if (!wait_r(bar(JOB_FULL + j), (seq >> 2) & 1)) break;
+      Job *jb = job(j);
+      if (jb->stop) break;
+      const int s = seq & 1, cbeg = jb->cbeg, n = jb->n, h = jb->h;
+      if (!wait_r(bar(SO + s), (seq >> 1) & 1)) break;
+      tc_fence_after();
+      const bool valid = i < n && cbeg + i < Tact;
+      __nv_bfloat16 *o = p.out + ((size_t)(cbeg + i) * p.H + h) * D;
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        uint32_t v[64];
+        tmem_ld64(tle + (s ? T_X1 : T_X0) + 64 * b, v);
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(v[8 * q + u]);
+            *reinterpret_cast<uint4 *>(o + 64 * b + 8 * q) = pack8(f);
+          }
+        }
+      }
+      tc_fence_before();
+      role_sync(BAR_EPI, 64);
+      if (i == 0) {
+        mbar_arrive(bar(XFREE + s));
+        mbar_arrive(bar(JOB_FREE + j));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *vabort) set_status(x.status, FLIDE_ERR_TIMEOUT);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ---- host ------------------------------------------------------------------
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -885,7 +1692,8 @@ int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, con
   if (dev < 0 || dev >= 64 || !attr_set[f8][dev].load(std::memory_order_acquire)) {
     const cudaError_t e =
         f8 ? cudaFuncSetAttribute(gdn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
-           : cudaFuncSetAttribute(gdn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+           : cudaFuncSetAttribute(gdn_ws_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ws::SMEM_BYTES);
     if (e != cudaSuccess) return FLIDE_ERR_CUDA;
     if (dev >= 0 && dev < 64) attr_set[f8][dev].store(true, std::memory_order_release);
   }
@@ -909,7 +1717,7 @@ int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, con
     if (f8)
       gdn_tc_kernel<true><<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
     else
-      gdn_tc_kernel<false><<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
+      gdn_ws_kernel<false><<<sms, ws::kThreads, ws::SMEM_BYTES, s>>>(mq, mk, mv, prm);
     FLIDE_LAUNCH_CHECK();
   }
   return FLIDE_OK;

@@ -143,12 +143,13 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
   const int A = block_scan_array(N, [&](int i) { return (int)x.depth[i] + 1; }, x.anc_ptr, scratch);
   (void)A;
   // ancestor rows (root first) and context lengths
+  const long long anc_cap = (long long)x.N * (x.max_depth + 1);
   for (int n = tid; n < N; n += blockDim.x) {
     int r = x.node_req[n], base = rp[r];
     int row = x.anc_ptr[n];
     int cur = n, ctx = d.past_len[r];
     for (int i = x.depth[n]; i >= 0; --i) {
-      x.anc_node[row + i] = cur;
+      if (in_bounds(x.status, x.counts, (long long)row + i, anc_cap, 101)) x.anc_node[row + i] = cur;
       ctx += d.seg_len[cur];
       if (i > 0) cur = base + d.parent[cur];
     }
@@ -165,7 +166,8 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
       int f = (n < N && x.depth[n] == lvl) ? 1 : 0;
       int tot;
       int ex = block_excl_scan(f, scratch, &tot);
-      if (f) x.level_node[placed + carry + ex] = n;
+      if (f && in_bounds(x.status, x.counts, placed + carry + ex, x.N, 102))
+        x.level_node[placed + carry + ex] = n;
       carry += tot;
     }
     placed += carry;
@@ -182,7 +184,8 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
   __syncthreads();
   for (int n = tid; n < N; n += blockDim.x) {
     int p = d.parent[n];
-    if (p >= 0) x.state_slot[rp[x.node_req[n]] + p] = 1;  // has children
+    if (p >= 0 && in_bounds(x.status, x.counts, rp[x.node_req[n]] + p, N, 103))
+      x.state_slot[rp[x.node_req[n]] + p] = 1;  // has children
   }
   __syncthreads();
   // inner nodes per level (L >= 1), for the two regions' sizes
@@ -192,7 +195,7 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
     int cnt = 0;
     for (int b = a0; b < a1; b += blockDim.x) {
       const int k = b + tid;
-      const int f = (k < a1 && x.state_slot[x.level_node[k]] == 1) ? 1 : 0;
+      const int f = (k < a1 && x.state_slot[checked(x.status, x.counts, x.level_node[k], N, 104)] == 1) ? 1 : 0;
       int tot;
       block_excl_scan(f, scratch, &tot);
       cnt += tot;
@@ -207,7 +210,7 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
       const int k = b + tid;
       int tot;
       const int ex = block_excl_scan(k < a1 ? 1 : 0, scratch, &tot);
-      if (k < a1) x.state_slot[x.level_node[k]] = roots + ex;
+      if (k < a1) x.state_slot[checked(x.status, x.counts, x.level_node[k], N, 105)] = roots + ex;
       roots += tot;
     }
   }
@@ -217,7 +220,7 @@ tree_nodes_kernel(flide_tree_desc d, flide_tree_index x) {
     int carry = 0;
     for (int b = a0; b < a1; b += blockDim.x) {
       const int k = b + tid;
-      const int n = k < a1 ? x.level_node[k] : -1;
+      const int n = k < a1 ? (int)checked(x.status, x.counts, x.level_node[k], N, 106) : -1;
       const int f = (n >= 0 && x.state_slot[n] == 1) ? 1 : 0;
       int tot;
       const int ex = block_excl_scan(f, scratch, &tot);
@@ -262,6 +265,7 @@ __global__ void tree_tokens_kernel(flide_tree_index x) {
     int n = upper_bound(x.node_start, N + 1, t) - 1;
     // nodes with zero tokens share a start with their successor; upper_bound
     // already picks the last node starting at or before t, which holds t.
+    if (!in_bounds(x.status, x.counts, n, N, 107)) continue;
     x.token_node[t] = n;
     x.token_pos[t] = x.ctx_len[n] - (x.node_start[n + 1] - x.node_start[n]) + (t - x.node_start[n]);
   }

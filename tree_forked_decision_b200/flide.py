@@ -13,13 +13,16 @@ import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libflide.so")
+# FLIDE_DEBUG_BOUNDS=1 selects the bounds-checked build (build.py --debug-bounds)
+LIB_PATH = os.path.join(_PKG, "libflide_dbg.so" if os.environ.get("FLIDE_DEBUG_BOUNDS") == "1"
+                        else "libflide.so")
 
-OK, ERR_INVALID, ERR_SHAPE, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID, ERR_SHAPE, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(7)
 F32, BF16, E4M3 = 0, 1, 2
 FLAG_PORTABLE = 1
 COUNTS = 16
-CNT = dict(N=0, T=1, PAST=2, DEPTH=3, SLOTS=4, BRANCH_TOK=5, ROOT_TOK=6, CKPT_ROWS=7)
+CNT = dict(N=0, T=1, PAST=2, DEPTH=3, SLOTS=4, BRANCH_TOK=5, ROOT_TOK=6, CKPT_ROWS=7,
+           CHECK_SITE=12, CHECK_VALUE=13)
 
 # names and order of the int32* members of flide_tree_index
 INDEX_ARRAYS = ["status", "counts", "node_start", "node_req", "depth", "anc_ptr", "anc_node",
@@ -35,7 +38,7 @@ SYMBOLS = ["flide_tree_index_bytes", "flide_tree_index_init", "flide_tree_build"
            "flide_history_append", "flide_history_gather", "flide_selftest_wait_timeout",
            "flide_fork_attn_fp8", "flide_amax", "flide_quantize_e4m3", "flide_fork_attn_paged",
            "flide_plan_state_groups", "flide_copy_rows", "flide_fork_gdn_fp8", "flide_pool_append_batch",
-           "flide_tree_state_slots", "flide_strerror"]
+           "flide_tree_state_slots", "flide_debug_bounds", "flide_strerror"]
 
 
 class FlideError(RuntimeError):
@@ -136,6 +139,8 @@ def _lib():
         lib.flide_amax.restype = ctypes.c_int
         lib.flide_quantize_e4m3.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
         lib.flide_quantize_e4m3.restype = ctypes.c_int
+        lib.flide_debug_bounds.argtypes = []
+        lib.flide_debug_bounds.restype = ctypes.c_int32
         lib.flide_strerror.argtypes = [ctypes.c_int32]
         lib.flide_strerror.restype = ctypes.c_char_p
         _LIB = lib
