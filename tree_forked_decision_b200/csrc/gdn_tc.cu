@@ -835,9 +835,9 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 //   S = gamma_last S0 + Delta'^T K               (Delta' = Delta gamma_last / gamma)
 // With gamma folded into Q's rows the output needs no second accumulator; the
 // extra rounding is one bf16 rounding of gamma_i q_i, like the bf16 copy of S0.
-// Roles (384 threads): warps 0-3 chain (TMEM lanes 0-127), 4-7 prep, 8 producer
-// (items, per-token scalars, TMA), 10-11 epilogue (output rows, TMEM lanes
-// 64-127); warp 9 idles.  The producer runs ahead through a ring of four chunk
+// Roles (384 threads): warps 0-3 prep, 4 producer (items, per-token scalars,
+// TMA), 6-7 epilogue (output rows, TMEM lanes 64-127), 8-11 chain (TMEM lanes
+// 0-127); warp 5 idles.  A warp reaches TMEM lanes 32 (w % 4) .. +31.  The producer runs ahead through a ring of four chunk
 // jobs, so the pipeline flows across items: a new item's first chunk starts
 // from its parent's state (global) while the previous item drains.  Every
 // handshake is an mbarrier whose next phase can only complete after its waiter
@@ -848,7 +848,13 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 namespace ws {
 
 constexpr int kThreads = 384;
-constexpr int kPrepWarp0 = 4, kProducerWarp = 8, kEpiWarp0 = 10;
+// Role of each warp.  A sub-partition (warps w, w+4, w+8) favours its lower
+// warp index when several warps can issue, so the critical prep warpgroup
+// takes the lowest indices and the producer, whose gate scan must keep ahead
+// of it, the next; the chain and the epilogue have slack.  (With the chain
+// below the prep and the producer, the producer's 64-token scan took 9K
+// cycles instead of under 1K.)
+constexpr int kPrepWarp0 = 0, kProducerWarp = 4, kEpiWarp0 = 6, kChainWarp0 = 8;
 constexpr int BAR_PREP = 1, BAR_CHAIN = 2, BAR_EPI = 3;  // named barriers
 
 // shared-memory map, bytes from a 1024-aligned base
@@ -866,7 +872,7 @@ constexpr int JOB_BYTES = 1600;
 constexpr int BARS = JOB + 4 * JOB_BYTES;
 enum {
   KQ_FULL = 0, KQ_EMPTY = 2, V_FULL = 4, V_EMPTY = 5, JOB_FULL = 6, JOB_FREE = 10, GRAM = 14,
-  WU = 15, READY = 16, CA_FREE = 17, XDONE = 18, SO = 19, XFREE = 21, DRAIN_P = 23,
+  WU = 15, READY = 16, CA_FREE = 17, XDONE = 18, SO = 19, XFREE = 21, DRAIN_P = 23,  // SO: 2
   DRAIN_C = 24, CK_FREE = 25, NBARS = 26
 };
 constexpr int MISC = BARS + 8 * NBARS;  // TMEM address, abort flag
@@ -875,7 +881,9 @@ static_assert(JOB % 16 == 0 && BARS % 8 == 0, "job slots and barriers must be al
 static_assert(SMEM_BYTES <= 232448, "shared memory over the 227 KB limit");
 
 // TMEM columns
-constexpr uint32_t T_S = 0, T_X0 = 128, T_X1 = 256, T_G = 384;
+// S: state; X: [U; 0] -> [Delta; gamma Q S0^T] -> outputs; G: [Q;K][Q;K]^T,
+// written for chunk c+1 while chunk c is solved; W: T' K
+constexpr uint32_t T_S = 0, T_X = 128, T_G = 256, T_W = 384;
 
 // One chunk of one (item, head), written by the producer: header, beta, the
 // segmented log2 decay G2, gamma = 2^G2, the separable decay factors
@@ -925,6 +933,65 @@ __device__ __forceinline__ void mma16x8(float (&acc)[4], FX X, FY Y, int lane) {
   for (int kk = 0; kk < 16; kk += 8) {
     mma_tf32_16x8x8(acc, to_tf32(X(g, kk + t)), to_tf32(X(g + 8, kk + t)), to_tf32(X(g, kk + t + 4)),
                     to_tf32(X(g + 8, kk + t + 4)), to_tf32(Y(kk + t, g)), to_tf32(Y(kk + t + 4, g)));
+  }
+}
+
+// Per-token scalars of one chunk into its job, one warp, two consecutive
+// tokens (t0 = 2 lane, t0 + 1) per lane: the segmented inclusive scan of g
+// (segments = the nodes of a packed group; s0/s1 = segment ids, -1 past the
+// chunk), G2 = log2 decay, gamma, the separable factors, the state-update
+// scales gamma_last / gamma_j and each token's segment start.  Kept out of
+// line: inlined into the producer loop its shuffle chain was scheduled badly.
+__device__ __noinline__ void gate_scan(Job *jb, int lane, int n, float b0, float b1, float a0,
+                                       float a1, int s0, int s1) {
+  const int t0 = 2 * lane, t1 = t0 + 1;
+  const bool v0 = s0 >= 0, v1 = s1 >= 0;
+  const int prev_s1 = __shfl_up_sync(0xffffffffu, s1, 1);
+  const bool cont0 = lane > 0 && prev_s1 == s0;  // token t0 continues token t0 - 1
+  float v = (s1 == s0) ? a0 + a1 : a1;
+  int f = (s1 != s0 || !cont0) ? 1 : 0;
+  const int st0 = cont0 ? -1 : t0, st1 = (s1 == s0) ? -1 : t1;  // segment starts
+  int m = max(st0, st1);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float pv = __shfl_up_sync(0xffffffffu, v, o);
+    const int pf = __shfl_up_sync(0xffffffffu, f, o);
+    const int pm = __shfl_up_sync(0xffffffffu, m, o);
+    if (lane >= o) {
+      if (!f) v += pv;
+      f |= pf;
+      m = max(m, pm);
+    }
+  }
+  const float carry = __shfl_up_sync(0xffffffffu, v, 1);
+  const int mprev = __shfl_up_sync(0xffffffffu, m, 1);
+  const int lo0 = max(lane > 0 ? mprev : -1, st0), lo1 = max(lo0, st1);
+  const float G0 = a0 + (cont0 ? carry : 0.f);
+  const float g0 = G0 * 1.4426950408889634f;
+  const float g1 = ((s1 == s0) ? G0 + a1 : a1) * 1.4426950408889634f;
+  float mx = fmaxf(v0 ? g0 : -INFINITY, v1 ? g1 : -INFINITY);
+  float mn = fminf(v0 ? g0 : INFINITY, v1 ? g1 : INFINITY);
+  mx = warp_max(mx);
+  mn = -warp_max(-mn);
+  const bool sep = !(mx - mn > 100.f);  // also true when no token is valid
+  const float gref = (mx >= mn) ? 0.5f * (mx + mn) : 0.f;
+  const float glast = __shfl_sync(0xffffffffu, (n - 1) & 1 ? g1 : g0, (n - 1) >> 1);
+  jb->beta[t0] = b0;
+  jb->beta[t1] = b1;
+  jb->g2[t0] = g0;
+  jb->g2[t1] = g1;
+  jb->gam[t0] = ex2_approx(g0);
+  jb->gam[t1] = ex2_approx(g1);
+  jb->f[t0] = sep ? ex2_approx(gref - g0) : 0.f;
+  jb->f[t1] = sep ? ex2_approx(gref - g1) : 0.f;
+  jb->dsc[t0] = v0 ? ex2_approx(glast - g0) : 0.f;
+  jb->dsc[t1] = v1 ? ex2_approx(glast - g1) : 0.f;
+  jb->lo[t0] = v0 ? lo0 : C;
+  jb->lo[t1] = v1 ? lo1 : C;
+  if (lane == 0) {
+    jb->gam_last = ex2_approx(glast);
+    jb->gref = gref;
+    jb->sep = sep ? 1 : 0;
   }
 }
 
@@ -990,6 +1057,23 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       jb = job(seq & 3);
       return true;
     };
+    // V of the previous chunk (issued one chunk behind its K and Q)
+    bool pend_v = false;
+    uint32_t pv_seq = 0;
+    int pv_cbeg = 0, pv_h = 0;
+    auto issue_v = [&]() -> bool {
+      if (!pend_v) return true;
+      if (!wait_w(bar(V_EMPTY), (pv_seq & 1) ^ 1)) return false;
+      if (lane == 0) {
+        const uint32_t vb = sb + V, fb = bar(V_FULL);
+        mbar_arrive_expect_tx(fb, 16384);
+        tma_load_3d(vb, &tm_v, fb, 0, pv_h, pv_cbeg);
+        tma_load_3d(vb + 8192, &tm_v, fb, 64, pv_h, pv_cbeg);
+      }
+      last_v = (int)pv_seq;
+      pend_v = false;
+      return true;
+    };
     for (;;) {
       unsigned long long it = 0;
       if (lane == 0) it = (unsigned long long)atomicAdd(groups_next(x, p.goff), 1);
@@ -1043,6 +1127,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
       if (stop) {
+        if (!issue_v()) { ok = false; break; }
         Job *jb;
         if (!claim(jb)) { ok = false; break; }
         if (lane == 0) jb->stop = 1;
@@ -1068,18 +1153,16 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!claim(jb)) { ok = false; break; }
         const int cbeg = tbeg + c * C;
         const int n = min(C, tend - cbeg);
-        // K and Q into stage s first, so the copy overlaps the scalar work
-        const int s = seq & 1;
-        if (!wait_w(bar(KQ_EMPTY + s), ((seq >> 1) & 1) ^ 1)) { ok = false; break; }
-        if (lane == 0) {
-          const uint32_t kq = sb + KQ + s * 32768, fb = bar(KQ_FULL + s);
-          mbar_arrive_expect_tx(fb, 32768);
-          tma_load_3d(kq, &tm_q, fb, 0, h, cbeg);
-          tma_load_3d(kq + 16384, &tm_q, fb, 64, h, cbeg);
-          tma_load_3d(kq + 8192, &tm_k, fb, 0, h, cbeg);
-          tma_load_3d(kq + 16384 + 8192, &tm_k, fb, 64, h, cbeg);
-        }
-        last_kq[s] = (int)(seq >> 1);
+        // the job first: per-token scalars and the gate scan, as soon as the
+        // slot is free, so the scan (slow next to the prep's shared-memory
+        // traffic) is done long before the prep starts this chunk
+        const int t0 = 2 * lane, t1 = t0 + 1;
+        const bool v0 = t0 < n && cbeg + t0 < Tact, v1 = t1 < n && cbeg + t1 < Tact;
+        const size_t i0 = (size_t)(cbeg + t0) * p.H + h, i1 = i0 + p.H;
+        const float b0 = v0 ? p.beta[i0] : 0.f, b1 = v1 ? p.beta[i1] : 0.f;
+        const float a0 = v0 ? p.g[i0] : 0.f, a1 = v1 ? p.g[i1] : 0.f;
+        const int s0 = v0 ? x.token_node[cbeg + t0] - n0 : -1;
+        const int s1 = v1 ? x.token_node[cbeg + t1] - n0 : -1;
         if (lane == 0) {
           jb->stop = 0;
           jb->cbeg = cbeg;
@@ -1091,76 +1174,28 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           jb->src = src;
           jb->dst = dst;
         }
-        {
-          // per-token scalars, two consecutive tokens per lane, and the
-          // segmented inclusive scan of g (segments = nodes of a packed group)
-          const int t0 = 2 * lane, t1 = t0 + 1;
-          const bool v0 = t0 < n && cbeg + t0 < Tact, v1 = t1 < n && cbeg + t1 < Tact;
-          const size_t i0 = (size_t)(cbeg + t0) * p.H + h, i1 = i0 + p.H;
-          const float b0 = v0 ? p.beta[i0] : 0.f, b1 = v1 ? p.beta[i1] : 0.f;
-          const float a0 = v0 ? p.g[i0] : 0.f, a1 = v1 ? p.g[i1] : 0.f;
-          const int s0 = v0 ? x.token_node[cbeg + t0] - n0 : -1;
-          const int s1 = v1 ? x.token_node[cbeg + t1] - n0 : -1;
-          const int prev_s1 = __shfl_up_sync(0xffffffffu, s1, 1);
-          const bool cont0 = lane > 0 && prev_s1 == s0;  // token t0 continues token t0 - 1
-          float v = (s1 == s0) ? a0 + a1 : a1;
-          int f = (s1 != s0 || !cont0) ? 1 : 0;
-          // segment starts: the latest start at or before each token
-          const int st0 = cont0 ? -1 : t0, st1 = (s1 == s0) ? -1 : t1;
-          int m = max(st0, st1);
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float pv = __shfl_up_sync(0xffffffffu, v, o);
-            const int pf = __shfl_up_sync(0xffffffffu, f, o);
-            const int pm = __shfl_up_sync(0xffffffffu, m, o);
-            if (lane >= o) {
-              if (!f) v += pv;
-              f |= pf;
-              m = max(m, pm);
-            }
-          }
-          const float carry = __shfl_up_sync(0xffffffffu, v, 1);
-          const int mprev = __shfl_up_sync(0xffffffffu, m, 1);
-          const int lo0 = max(lane > 0 ? mprev : -1, st0), lo1 = max(lo0, st1);
-          const float G0 = a0 + (cont0 ? carry : 0.f);
-          const float g0 = G0 * 1.4426950408889634f;
-          const float g1 = ((s1 == s0) ? G0 + a1 : a1) * 1.4426950408889634f;
-          float mx = fmaxf(v0 ? g0 : -INFINITY, v1 ? g1 : -INFINITY);
-          float mn = fminf(v0 ? g0 : INFINITY, v1 ? g1 : INFINITY);
-          mx = warp_max(mx);
-          mn = -warp_max(-mn);
-          const bool sep = !(mx - mn > 100.f);  // also true when no token is valid
-          const float gref = (mx >= mn) ? 0.5f * (mx + mn) : 0.f;
-          const float glast = __shfl_sync(0xffffffffu, (n - 1) & 1 ? g1 : g0, (n - 1) >> 1);
-          jb->beta[t0] = b0;
-          jb->beta[t1] = b1;
-          jb->g2[t0] = g0;
-          jb->g2[t1] = g1;
-          jb->gam[t0] = ex2_approx(g0);
-          jb->gam[t1] = ex2_approx(g1);
-          jb->f[t0] = sep ? ex2_approx(gref - g0) : 0.f;
-          jb->f[t1] = sep ? ex2_approx(gref - g1) : 0.f;
-          jb->dsc[t0] = v0 ? ex2_approx(glast - g0) : 0.f;
-          jb->dsc[t1] = v1 ? ex2_approx(glast - g1) : 0.f;
-          jb->lo[t0] = v0 ? lo0 : C;
-          jb->lo[t1] = v1 ? lo1 : C;
-          if (lane == 0) {
-            jb->gam_last = ex2_approx(glast);
-            jb->gref = gref;
-            jb->sep = sep ? 1 : 0;
-          }
-        }
+        gate_scan(jb, lane, n, b0, b1, a0, a1, s0, s1);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(JOB_FULL + (seq & 3)));
-        // V
-        if (!wait_w(bar(V_EMPTY), (seq & 1) ^ 1)) { ok = false; break; }
+        // then K and Q into stage s
+        const int s = seq & 1;
+        if (!wait_w(bar(KQ_EMPTY + s), ((seq >> 1) & 1) ^ 1)) { ok = false; break; }
         if (lane == 0) {
-          const uint32_t vb = sb + V, fb = bar(V_FULL);
-          mbar_arrive_expect_tx(fb, 16384);
-          tma_load_3d(vb, &tm_v, fb, 0, h, cbeg);
-          tma_load_3d(vb + 8192, &tm_v, fb, 64, h, cbeg);
+          const uint32_t kq = sb + KQ + s * 32768, fb = bar(KQ_FULL + s);
+          mbar_arrive_expect_tx(fb, 32768);
+          tma_load_3d(kq, &tm_q, fb, 0, h, cbeg);
+          tma_load_3d(kq + 16384, &tm_q, fb, 64, h, cbeg);
+          tma_load_3d(kq + 8192, &tm_k, fb, 0, h, cbeg);
+          tma_load_3d(kq + 16384 + 8192, &tm_k, fb, 64, h, cbeg);
         }
-        last_v = (int)seq;
+        last_kq[s] = (int)(seq >> 1);
+        // the previous chunk's V: its buffer frees when that chunk's prep
+        // has used the previous V, long before this point in steady state
+        if (!issue_v()) { ok = false; break; }
+        pend_v = true;
+        pv_seq = seq;
+        pv_cbeg = cbeg;
+        pv_h = h;
       }
       if (!ok) break;
     }
@@ -1184,21 +1219,21 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (pt == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
       return role_and(BAR_PREP, 128, r);
     };
-    for (uint32_t seq = 0;; ++seq) {
-      if (!wait_r(bar(JOB_FULL + (seq & 3)), (seq >> 2) & 1)) break;
-      Job *jb = job(seq & 3);
-      if (jb->stop) break;
-      const int n = jb->n, s = seq & 1;
-      const uint32_t kq = sb + KQ + s * 32768;
-      uint8_t *kqp = smem + KQ + s * 32768;
-      // -- 2. this chunk's Q and K; rows past the chunk's tokens zeroed (they
-      //       may hold another node's tokens or uninitialised memory)
-      if (!wait_r(bar(KQ_FULL + s), (seq >> 1) & 1)) break;
-      if (n < C) {
+    // A chunk's start: its job, its Q and K (rows past its tokens zeroed:
+    // they may hold another node's tokens or uninitialised memory) and its
+    // [Q;K][Q;K]^T into G.  1 = the producer's stop job, -1 = a wait gave up.
+    auto start_chunk = [&](uint32_t sq) -> int {
+      if (!wait_r(bar(JOB_FULL + (sq & 3)), (sq >> 2) & 1)) return -1;
+      const Job *jn = job(sq & 3);
+      if (jn->stop) return 1;
+      const int nn = jn->n, ss = sq & 1;
+      uint8_t *kqn = smem + KQ + ss * 32768;
+      if (!wait_r(bar(KQ_FULL + ss), (sq >> 1) & 1)) return -1;
+      if (nn < C) {
         for (int e = pt; e < 4 * C * 8; e += 128) {  // (slab, Q|K, row, 16-byte chunk)
           const int row = (e >> 3) & (C - 1);
-          if (row >= n)
-            *reinterpret_cast<uint4 *>(kqp + (e >> 10) * 16384 + ((e >> 9) & 1) * 8192 + row * 128 +
+          if (row >= nn)
+            *reinterpret_cast<uint4 *>(kqn + (e >> 10) * 16384 + ((e >> 9) & 1) * 8192 + row * 128 +
                                        (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
@@ -1206,16 +1241,25 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       role_sync(BAR_PREP, 128);
       if (pt == 0) {
         tc_fence_after();
+        const uint32_t kqa = sb + KQ + ss * 32768;
         constexpr uint32_t id = idesc_bf16(128, 128, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t d = sdesc_sw128(kq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t d = sdesc_sw128(kqa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           mma_bf16(tmem + T_G, d, d, id, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(GRAM));
         issued = true;
       }
       __syncwarp();
+      return 0;
+    };
+    int next = start_chunk(0);
+    for (uint32_t seq = 0; next == 0; ++seq) {
+      Job *jb = job(seq & 3);
+      const int n = jb->n, s = seq & 1;
+      const uint32_t kq = sb + KQ + s * 32768;
+      uint8_t *kqp = smem + KQ + s * 32768;
       if (!wait_r(bar(GRAM), seq & 1)) break;
       tc_fence_after();
       // -- 3. decay masks from the Gram columns 64-127 (k_j): rows 0-63 are
@@ -1253,7 +1297,11 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
         }
       }
+      tc_fence_before();
       role_sync(BAR_PREP, 128);
+      // the next chunk's job, Q, K and Gram, behind this chunk's solve
+      next = start_chunk(seq + 1);
+      if (next < 0) break;
       // -- 4. T = (I + A)^-1: the four diagonal 16 x 16 blocks by substitution,
       //       then the off-diagonal blocks by doubling: T_10, T_32 from
       //       T_ii (-A_ij) T_jj, then the lower-left 32 x 32 block the same way
@@ -1357,8 +1405,8 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           st_chunk(t2, i, 4 * half + q, pack8(f2));
         }
       }
-      // -- 6. V (rows past the chunk zeroed), then W = T' K -> T_G and
-      //       U = [T''; 0] V -> X[s] once the epilogue of chunk seq-2 has read X[s]
+      // -- 6. V (rows past the chunk zeroed), then W = T' K -> W and
+      //       U = [T''; 0] V -> X once the epilogue of chunk seq-1 has read X
       if (!wait_r(bar(V_FULL), seq & 1)) break;
       if (n < C) {
         for (int e = pt; e < 2 * C * 8; e += 128) {
@@ -1369,14 +1417,14 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
       fence_proxy_async_smem();
-      if (!wait_r(bar(XFREE + s), ((seq >> 1) & 1) ^ 1)) break;
+      if (!wait_r(bar(XFREE), (seq & 1) ^ 1)) break;
       if (pt == 0) {
         tc_fence_after();
         constexpr uint32_t id = idesc_bf16(128, 128, true);
-        const uint32_t xs_t = tmem + (s ? T_X1 : T_X0);
+        const uint32_t xs_t = tmem + T_X;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16(tmem + T_G, sdesc_sw128(sb + TT + kk * 32, 16, 1024),
+          mma_bf16(tmem + T_W, sdesc_sw128(sb + TT + kk * 32, 16, 1024),
                    sdesc_sw128(kq + 8192 + kk * 2048, 16384, 1024), id, kk > 0 ? 1u : 0u);
           mma_bf16(xs_t, sdesc_sw128(sb + TT + 8192 + kk * 32, 16, 1024),
                    sdesc_sw128(sb + V + kk * 2048, 8192, 1024), id, kk > 0 ? 1u : 0u);
@@ -1395,7 +1443,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
           uint32_t w[64];
-          tmem_ld64(tlp + T_G + 64 * b, w);
+          tmem_ld64(tlp + T_W + 64 * b, w);
           uint8_t *dst = smem + CA + b * 16384;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -1444,14 +1492,14 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mma_commit(bar(DRAIN_P));
       mbar_wait(bar(DRAIN_P), 0, vabort, kTimeoutNs, false);
     }
-  } else if (warp < 4) {
+  } else if (warp >= kChainWarp0) {
     // ---------------- chain: the state products, chunk after chunk
-    const int row = tid;  // TMEM lane = state row (dv) / token row
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const int row = tid - kChainWarp0 * 32;  // TMEM lane = state row (dv) / token row
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     bool issued = false;
     auto wait_r = [&](uint32_t b, uint32_t parity) -> bool {  // one poller, the rest park
       bool r = true;
-      if (tid == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
+      if (row == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
       return role_and(BAR_CHAIN, 128, r);
     };
     for (uint32_t seq = 0;; ++seq) {
@@ -1465,7 +1513,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       float *dst = jb->dst;
       if (!wait_r(bar(READY), seq & 1)) break;
       const float gl = jb->gam_last;
-      const uint32_t xt = s ? T_X1 : T_X0;
+      const uint32_t xt = T_X;
       // -- S0 as the bf16 B operand; S <- gamma_last S for the update
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
@@ -1500,7 +1548,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       fence_proxy_async_smem();
       tc_fence_before();
       role_sync(BAR_CHAIN, 128);
-      if (tid == 0) {
+      if (row == 0) {
         tc_fence_after();
         constexpr uint32_t id = idesc_bf16(128, 128, false);
 #pragma unroll
@@ -1515,7 +1563,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __syncwarp();
       if (!wait_r(bar(XDONE), seq & 1)) break;
       tc_fence_after();
-      if (tid == 0) mbar_arrive(bar(CA_FREE));
+      if (row == 0) mbar_arrive(bar(CA_FREE));
       // -- Delta (token rows 0-63) as the MN-major B of (M o QK^T) Delta, and
       //    Delta' = Delta gamma_last / gamma_j as the MN-major A of the update
       if (row < C) {
@@ -1540,7 +1588,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       fence_proxy_async_smem();
       tc_fence_before();
       role_sync(BAR_CHAIN, 128);
-      if (tid == 0) {
+      if (row == 0) {
         tc_fence_after();
         const uint32_t mq = sb + MQK + s * 8192 - 8192;  // [junk; M o QK^T]
 #pragma unroll
@@ -1557,7 +1605,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __syncwarp();
       if (!wait_r(bar(SO + s), (seq >> 1) & 1)) break;
       tc_fence_after();
-      if (tid == 0) {
+      if (row == 0) {
         mbar_arrive(bar(CK_FREE));
         mbar_arrive(bar(JOB_FREE + j));
       }
@@ -1575,11 +1623,11 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
     }
-    if (tid == 0 && issued && *vabort) {
+    if (row == 0 && issued && *vabort) {
       mma_commit(bar(DRAIN_C));
       mbar_wait(bar(DRAIN_C), 0, vabort, kTimeoutNs, false);
     }
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 2) {
     // ---------------- epilogue: output rows (TMEM lanes 64-127 of X)
     const int i = tid - kEpiWarp0 * 32;  // token of the chunk
     const uint32_t tle = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -1601,7 +1649,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         uint32_t v[64];
-        tmem_ld64(tle + (s ? T_X1 : T_X0) + 64 * b, v);
+        tmem_ld64(tle + T_X + 64 * b, v);
         if (valid) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -1615,7 +1663,7 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_before();
       role_sync(BAR_EPI, 64);
       if (i == 0) {
-        mbar_arrive(bar(XFREE + s));
+        mbar_arrive(bar(XFREE));
         mbar_arrive(bar(JOB_FREE + j));
       }
     }
