@@ -835,9 +835,10 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 //   S = gamma_last S0 + Delta'^T K               (Delta' = Delta gamma_last / gamma)
 // With gamma folded into Q's rows the output needs no second accumulator; the
 // extra rounding is one bf16 rounding of gamma_i q_i, like the bf16 copy of S0.
-// Roles (384 threads): warps 0-3 prep, 4 producer (items, per-token scalars,
-// TMA), 6-7 epilogue (output rows, TMEM lanes 64-127), 8-11 chain (TMEM lanes
-// 0-127); warp 5 idles.  A warp reaches TMEM lanes 32 (w % 4) .. +31.  The producer runs ahead through a ring of four chunk
+// Roles (512 threads): warps 0-7 prep (two per TMEM lane quadrant), 8
+// producer (items, per-token scalars, TMA), 10-11 epilogue (output rows, TMEM
+// lanes 64-127), 12-15 chain (TMEM lanes 0-127); warp 9 idles.  A warp reaches
+// TMEM lanes 32 (w % 4) .. +31.  The producer runs ahead through a ring of four chunk
 // jobs, so the pipeline flows across items: a new item's first chunk starts
 // from its parent's state (global) while the previous item drains.  Every
 // handshake is an mbarrier whose next phase can only complete after its waiter
@@ -847,14 +848,14 @@ gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // c's first product has read them, and copies K once c's update has.
 namespace ws {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 // Role of each warp.  A sub-partition (warps w, w+4, w+8) favours its lower
 // warp index when several warps can issue, so the critical prep warpgroup
 // takes the lowest indices and the producer, whose gate scan must keep ahead
 // of it, the next; the chain and the epilogue have slack.  (With the chain
 // below the prep and the producer, the producer's 64-token scan took 9K
 // cycles instead of under 1K.)
-constexpr int kPrepWarp0 = 0, kProducerWarp = 4, kEpiWarp0 = 6, kChainWarp0 = 8;
+constexpr int kPrepWarp0 = 0, kPrepWarps = 8, kProducerWarp = 8, kEpiWarp0 = 10, kChainWarp0 = 12;
 constexpr int BAR_PREP = 1, BAR_CHAIN = 2, BAR_EPI = 3;  // named barriers
 
 // shared-memory map, bytes from a 1024-aligned base
@@ -1206,18 +1207,24 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (last_v >= 0) mbar_wait(bar(V_FULL), last_v & 1, vabort, kTimeoutNs, false);
     }
     __syncwarp();
-  } else if (warp >= kPrepWarp0 && warp < kPrepWarp0 + 4) {
-    // ---------------- prep: everything of a chunk that does not need the state
-    const int pt = tid - kPrepWarp0 * 32;
+  } else if (warp >= kPrepWarp0 && warp < kPrepWarp0 + kPrepWarps) {
+    // ---------------- prep: everything of a chunk that does not need the state.
+    // Two warps per TMEM lane quadrant (warps w and w + 4); the second of each
+    // pair takes the other half of every column range.
+    const int pt = tid - kPrepWarp0 * 32;         // 0 .. 255
+    const int pw = warp - kPrepWarp0;             // 0 .. 7
+    const int hb = pw >> 2;                       // column half
+    const int row = (warp & 3) * 32 + lane;       // this thread's TMEM lane
     const uint32_t tlp = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     float *Pm = reinterpret_cast<float *>(smem + PM);
     float *Xs = reinterpret_cast<float *>(smem + TT);  // 4 blocks of 16 x 17 during the solve
     constexpr int XS_LD = 17;
+    constexpr int NP = 32 * kPrepWarps;
     bool issued = false;  // MMAs in flight (pt == 0), for the drain
     auto wait_r = [&](uint32_t b, uint32_t parity) -> bool {  // one poller, the rest park
       bool r = true;
       if (pt == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
-      return role_and(BAR_PREP, 128, r);
+      return role_and(BAR_PREP, NP, r);
     };
     // A chunk's start: its job, its Q and K (rows past its tokens zeroed:
     // they may hold another node's tokens or uninitialised memory) and its
@@ -1230,15 +1237,15 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       uint8_t *kqn = smem + KQ + ss * 32768;
       if (!wait_r(bar(KQ_FULL + ss), (sq >> 1) & 1)) return -1;
       if (nn < C) {
-        for (int e = pt; e < 4 * C * 8; e += 128) {  // (slab, Q|K, row, 16-byte chunk)
-          const int row = (e >> 3) & (C - 1);
-          if (row >= nn)
-            *reinterpret_cast<uint4 *>(kqn + (e >> 10) * 16384 + ((e >> 9) & 1) * 8192 + row * 128 +
+        for (int e = pt; e < 4 * C * 8; e += NP) {  // (slab, Q|K, row, 16-byte chunk)
+          const int r = (e >> 3) & (C - 1);
+          if (r >= nn)
+            *reinterpret_cast<uint4 *>(kqn + (e >> 10) * 16384 + ((e >> 9) & 1) * 8192 + r * 128 +
                                        (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
+        role_sync(BAR_PREP, NP);
       }
-      role_sync(BAR_PREP, 128);
       if (pt == 0) {
         tc_fence_after();
         const uint32_t kqa = sb + KQ + ss * 32768;
@@ -1267,38 +1274,39 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       //       (fp32, kept transposed above the diagonal of the solve area)
       {
         const bool sep = jb->sep != 0;
-        const bool qrow = pt < C;
-        const int i = pt & (C - 1);
+        const bool qrow = row < C;
+        const int i = row & (C - 1);
         const float G2i = jb->g2[i];
         const int lo = jb->lo[i], hi = qrow ? i : i - 1;  // visible j: lo <= j <= hi
         const float sc = qrow ? dsq * dsk : jb->beta[i] * (dsk * dsk);
         const float ei = sc * (sep ? ex2_approx(G2i - jb->gref) : 1.f);
-        uint32_t d[64];
-        tmem_ld64(tlp + T_G + 64, d);
+        uint32_t d[32];
+        tmem_ld32(tlp + T_G + 64 + 32 * hb, d);
         uint8_t *mq = smem + MQK + s * 8192;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {  // 8 columns at a time: few live registers
-          const float4 fa = reinterpret_cast<const float4 *>(sep ? jb->f : jb->g2)[2 * q];
-          const float4 fb = reinterpret_cast<const float4 *>(sep ? jb->f : jb->g2)[2 * q + 1];
+        for (int q = 0; q < 4; ++q) {  // 8 columns at a time
+          const int j0 = 32 * hb + 8 * q;
+          const float4 fa = reinterpret_cast<const float4 *>(sep ? jb->f : jb->g2)[j0 >> 2];
+          const float4 fb = reinterpret_cast<const float4 *>(sep ? jb->f : jb->g2)[(j0 >> 2) + 1];
           const float fj[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
           float e[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int j = 8 * q + u;
+            const int j = j0 + u;
             const float ratio = sep ? ei * fj[u] : ei * ex2_approx(G2i - fj[u]);
-            e[u] = (j >= lo && j <= hi) ? ratio * __uint_as_float(d[j]) : 0.f;
+            e[u] = (j >= lo && j <= hi) ? ratio * __uint_as_float(d[8 * q + u]) : 0.f;
           }
           if (qrow) {
-            st_chunk(mq, i, q, pack8(e));
+            st_chunk(mq, i, 4 * hb + q, pack8(e));
           } else {
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-              if (8 * q + u < i) Pm[(8 * q + u) * P_LD + i] = e[u];
+              if (j0 + u < i) Pm[(j0 + u) * P_LD + i] = e[u];
           }
         }
       }
       tc_fence_before();
-      role_sync(BAR_PREP, 128);
+      role_sync(BAR_PREP, NP);
       // the next chunk's job, Q, K and Gram, behind this chunk's solve
       next = start_chunk(seq + 1);
       if (next < 0) break;
@@ -1323,16 +1331,15 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int i = 0; i < 16; ++i)
           if (i > cc) Pm[(r0 + i) * P_LD + r0 + cc] = tcol[i];
       }
-      role_sync(BAR_PREP, 128);
-      {
-        // T_10 (warps 4, 5: column halves) and T_32 (warps 6, 7)
-        const int wq = warp - kPrepWarp0;
-        const int I = (wq >> 1) ? 3 : 1, J = I - 1, half = wq & 1;
+      role_sync(BAR_PREP, NP);
+      if (pw < 4) {
+        // T_10 (warps 0, 1: column halves) and T_32 (warps 2, 3)
+        const int I = (pw >> 1) ? 3 : 1, J = I - 1, half = pw & 1;
         const int rI = 16 * I, cJ = 16 * J, cn = cJ + 8 * half;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         mma16x8(acc, [&](int r, int k) { return a_at(Pm, rI + r, cJ + k); },
                 [&](int k, int c) { return t_at(Pm, cJ + k, cn + c); }, lane);
-        float *xs = Xs + wq * 16 * XS_LD;
+        float *xs = Xs + pw * 16 * XS_LD;
         const int g = lane >> 2, t = lane & 3;
         xs[g * XS_LD + 2 * t] = acc[0];
         xs[g * XS_LD + 2 * t + 1] = acc[1];
@@ -1347,16 +1354,16 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         Pm[(rI + g + 8) * P_LD + cn + 2 * t] = -acc2[2];
         Pm[(rI + g + 8) * P_LD + cn + 2 * t + 1] = -acc2[3];
       }
-      role_sync(BAR_PREP, 128);
+      role_sync(BAR_PREP, NP);
       {
         // lower-left 32 x 32: X_IJ = sum_{K=J..1} A_IK T_KJ, then
-        // T_IJ = -sum_{K=2..I} T_IK X_KJ; warp (I, J) = 4:(2,0) 5:(2,1) 6:(3,0) 7:(3,1)
-        const int wq = warp - kPrepWarp0;
-        const int I = 2 + (wq >> 1), J = wq & 1;
+        // T_IJ = -sum_{K=2..I} T_IK X_KJ; block (I, J) = (2 + (b >> 1), b & 1)
+        // for b = pw >> 1, column tile nt = pw & 1 of it
+        const int blk = pw >> 1, nt = pw & 1;
+        const int I = 2 + (blk >> 1), J = blk & 1;
         const int g = lane >> 2, t = lane & 3;
-        float *xs = Xs + wq * 16 * XS_LD;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        float *xs = Xs + blk * 16 * XS_LD;
+        {
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int K = 0; K <= 1; ++K)
@@ -1368,9 +1375,8 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           xs[(g + 8) * XS_LD + 8 * nt + 2 * t] = acc[2];
           xs[(g + 8) * XS_LD + 8 * nt + 2 * t + 1] = acc[3];
         }
-        role_sync(BAR_PREP, 128);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        role_sync(BAR_PREP, NP);
+        {
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int K = 2; K <= 3; ++K) {
@@ -1386,33 +1392,33 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           Pm[(16 * I + g + 8) * P_LD + cn + 2 * t + 1] = -acc[3];
         }
       }
-      role_sync(BAR_PREP, 128);
+      role_sync(BAR_PREP, NP);
       // -- 5. T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles
       {
-        const int i = pt >> 1, half = pt & 1;
+        const int i = pt >> 2, qq = pt & 3;  // row, 16-column quarter
         uint8_t *t1 = smem + TT, *t2 = smem + TT + 8192;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           float f1[8], f2[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int j = 32 * half + 8 * q + u;
+            const int j = 16 * qq + 8 * q + u;
             const float tv = t_at(Pm, i, j), b = jb->beta[j];
             f1[u] = tv * (b * jb->gam[j] * dsk);
             f2[u] = tv * (b * dsv);
           }
-          st_chunk(t1, i, 4 * half + q, pack8(f1));
-          st_chunk(t2, i, 4 * half + q, pack8(f2));
+          st_chunk(t1, i, 2 * qq + q, pack8(f1));
+          st_chunk(t2, i, 2 * qq + q, pack8(f2));
         }
       }
       // -- 6. V (rows past the chunk zeroed), then W = T' K -> W and
       //       U = [T''; 0] V -> X once the epilogue of chunk seq-1 has read X
       if (!wait_r(bar(V_FULL), seq & 1)) break;
       if (n < C) {
-        for (int e = pt; e < 2 * C * 8; e += 128) {
-          const int row = (e >> 3) & (C - 1);
-          if (row >= n)
-            *reinterpret_cast<uint4 *>(smem + V + (e >> 9) * 8192 + row * 128 + (e & 7) * 16) =
+        for (int e = pt; e < 2 * C * 8; e += NP) {
+          const int r = (e >> 3) & (C - 1);
+          if (r >= n)
+            *reinterpret_cast<uint4 *>(smem + V + (e >> 9) * 8192 + r * 128 + (e & 7) * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
         }
       }
@@ -1435,54 +1441,53 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!wait_r(bar(WU), seq & 1)) break;
       tc_fence_after();
       if (pt == 0) mbar_arrive(bar(V_EMPTY));
-      // -- 7. the chain's tiles, each once chunk seq-1's chain has finished
-      //       with it: [-W; gamma Q] after its first product, K after the update
-      if (!wait_r(bar(CA_FREE), (seq & 1) ^ 1)) break;
-      if (pt < C) {
-        const int i = pt;  // W row = token (TMEM lanes 0-63)
+      // -- 7. the chain's tiles, once chunk seq-1's chain has finished with
+      //       them: [-W; gamma Q] (read by its first product) and K (by its
+      //       update); both are long free when the prep is the slower role
+      if (pt == 0) {
+        bool r = mbar_wait(bar(CA_FREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
+        r = r && mbar_wait(bar(CK_FREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
+        if (!r) *vabort = 1;
+      }
+      if (!role_and(BAR_PREP, NP, *vabort == 0 || pt != 0)) break;
+      if (row < C) {
+        // W row = token (TMEM lanes 0-63), dk half hb
+        uint32_t w[64];
+        tmem_ld64(tlp + T_W + 64 * hb, w);
+        uint8_t *dst = smem + CA + hb * 16384;
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          uint32_t w[64];
-          tmem_ld64(tlp + T_W + 64 * b, w);
-          uint8_t *dst = smem + CA + b * 16384;
+        for (int q = 0; q < 8; ++q) {
+          float f[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float f[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(w[8 * q + u]);
-            st_chunk(dst, i, q, pack8(f));
-          }
+          for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(w[8 * q + u]);
+          st_chunk(dst, row, q, pack8(f));
         }
       } else {
-        const int i = pt - C;  // gamma_i q_i into tile rows 64-127 (same swizzle phase)
+        const int i = row - C;  // gamma_i q_i into tile rows 64-127 (same swizzle phase), dk half hb
         const float gq = jb->gam[i] * dsq;
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int q = 0; q < 8; ++q) {
+          const int off = i * 128 + ((q ^ (i & 7)) << 4);
+          const uint4 raw = *reinterpret_cast<const uint4 *>(kqp + hb * 16384 + off);
+          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+          float f[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int off = i * 128 + ((q ^ (i & 7)) << 4);
-            const uint4 raw = *reinterpret_cast<const uint4 *>(kqp + b * 16384 + off);
-            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-            float f[8];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[u]));
-              f[2 * u] = v2.x * gq;
-              f[2 * u + 1] = v2.y * gq;
-            }
-            *reinterpret_cast<uint4 *>(smem + CA + b * 16384 + 8192 + off) = pack8(f);
+          for (int u = 0; u < 4; ++u) {
+            const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[u]));
+            f[2 * u] = v2.x * gq;
+            f[2 * u + 1] = v2.y * gq;
           }
+          *reinterpret_cast<uint4 *>(smem + CA + hb * 16384 + 8192 + off) = pack8(f);
         }
       }
-      if (!wait_r(bar(CK_FREE), (seq & 1) ^ 1)) break;
-      for (int e = pt; e < 2 * C * 8; e += 128) {  // K rows: same rows, same swizzle
+      for (int e = pt; e < 2 * C * 8; e += NP) {  // K rows: same rows, same swizzle
         const int b = e >> 9, rest = (e & 511) * 16;
         *reinterpret_cast<uint4 *>(smem + CK + b * 8192 + rest) =
             *reinterpret_cast<const uint4 *>(kqp + b * 16384 + 8192 + rest);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      role_sync(BAR_PREP, 128);
+      role_sync(BAR_PREP, NP);
       if (pt == 0) {
         mbar_arrive(bar(READY));
         mbar_arrive(bar(KQ_EMPTY + s));
