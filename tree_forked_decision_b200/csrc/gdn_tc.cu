@@ -1,5 +1,5 @@
 // gdn_tc.cu -- Gated DeltaNet fork scan on the 5th-generation tensor cores
-// (sm_100a): bf16 q/k/v, dk = dv = 128, fp32 state and accumulation.
+// (sm_100a): bf16 or e4m3 q/k/v, dk = dv = 128, fp32 state and accumulation.
 //
 // Per head the state S (dv x dk) follows the gated delta rule
 //   S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t.
@@ -16,16 +16,10 @@
 //   W = T diag(b gamma) K,   U = T diag(b) V,   Delta = U - W S0^T,
 //   O = diag(gamma) Q S0^T + (M o QK^T) Delta,  M_ij = gamma_i/gamma_j (j <= i),
 //   S_end = gamma_last S0 + Delta^T diag(gamma_last/gamma) K.
-// Tensor-core products, all M = 128 x N = 128 with a K-major shared-memory A
-// operand (rows = tokens padded to 128, or state rows):
-//   R1 = [K;Q] [K;Q]^T     -> KK^T (rows 0-63) and QK^T (rows 64-127)
-//   R2 = T' K,  R3 = T'' V -> W and U (T' = T diag(b gamma), T'' = T diag(b))
-//   R3 += (-W) S0^T        -> Delta         R1 = [K;Q] S0^T -> Q S0^T (rows 64-127)
-//   R2 = (M o QK^T) Delta  -> rows 64-127   S += Delta'^T K  (Delta' = Delta gamma_last/gamma)
-// T is solved in fp32 on CUDA cores by 16 x 16 blocks: the four diagonal
-// blocks by substitution, then block row i from T_ij = -T_ii sum_k A_ik T_kj.
-// The fp32 state
-// lives in TMEM for the whole scan; a bf16 copy is the operand for a chunk.
+// Only the last three lines need the state; everything above them is a
+// function of the chunk's own inputs.  The kernel below (gdn_ws_kernel) runs
+// the two parts in different warps, chunk c+1's state-free part while chunk
+// c's state products run.
 //
 // Work items (built per level by gdn_groups_kernel): a root, an inner node or
 // a node longer than one chunk is a "scan" item (its chunks in order, state
@@ -49,32 +43,7 @@ using namespace sm100;
 
 constexpr int C = 64;    // tokens per chunk
 constexpr int D = 128;   // dk = dv
-constexpr int kThreads = 256;  // two warps per TMEM lane group: warp w and w + 4 split the columns
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-
-// shared-memory map, bytes from a 1024-aligned base
-constexpr int SM_KQ = 0;        // stage s: s*32768; slab b (64 dims): +b*16384; K rows 0-63, Q rows 64-127
-constexpr int SM_V = 65536;     // stage s: s*16384; slab b: +b*8192; rows 0-63
-constexpr int SM_S0 = 98304;    // bf16 S0 [128 dv rows][dk], K-major, 2 slabs x 16 KB; then
-                                //   Delta [64 token rows][dv] MN-major (2 slabs x 8 KB) at +0 and
-                                //   Delta'^T [128 dv rows][64 tokens] K-major at +16384
-constexpr int SM_TA = 131072;   // T' and T'' [128 rows][64] K-major (16 KB each); then
-                                //   -W [128 rows][dk] K-major (2 slabs x 16 KB)
-constexpr int SM_PM = 163840;   // (M o QK^T) [128 rows][64] K-major, token rows at 64-127
-constexpr int SM_A = 180224;    // fp32 A [64][65]
-constexpr int A_LD = 65;
-constexpr int SM_T = SM_A + C * A_LD * 4;     // fp32 T [64][65]
-constexpr int SM_X = SM_T + C * A_LD * 4;     // fp32 block products X [3][16][17]
-constexpr int X_LD = 17;
-constexpr int SM_SCAL = SM_X + 3 * 16 * X_LD * 4;  // beta, G, gamma, seg, G*log2(e): 5 x 64 words
-constexpr int SM_BAR = SM_SCAL + 5 * C * 4;
-constexpr int SM_MISC = SM_BAR + 64;
-constexpr int SMEM_BYTES = SM_MISC + 64 + 1024;
-
-// TMEM column regions (128 each)
-constexpr uint32_t R_S = 0, R1 = 128, R2 = 256, R3 = 384;
-
-enum { B_FULL = 0, B_MMA = 2, NUM_BARS = 3 };
 
 struct GdnTcParams {
   flide_tree_index x;
@@ -199,12 +168,6 @@ __device__ __forceinline__ void st_chunk(uint8_t *base, int row, int q, uint4 v)
   *reinterpret_cast<uint4 *>(base + row * 128 + ((q ^ (row & 7)) << 4)) = v;
 }
 
-// byte offset of element (row, col) in a K-major tile of 128-byte rows
-// (64 bf16 per row) with the 128-byte swizzle
-__device__ __forceinline__ uint32_t sw_elem(int row, int col) {
-  return row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2;
-}
-
 // 16 x 16 x 16 block products of the triangular solve on the warp's tensor
 // path: mma.sync m16n8k8 with tf32 inputs (rounded to nearest) and fp32
 // accumulation.  Fragments (g = lane / 4, t = lane % 4): A rows g, g+8 and
@@ -224,35 +187,6 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// acc += A (16 x 16, row stride lda) B (16 x 16, row stride ldb), fp32 in shared memory
-__device__ __forceinline__ void block_mma16(float (&acc)[2][4], const float *A, int lda, const float *B,
-                                            int ldb, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int kk = 0; kk < 16; kk += 8) {
-    const uint32_t a0 = to_tf32(A[g * lda + kk + t]), a1 = to_tf32(A[(g + 8) * lda + kk + t]);
-    const uint32_t a2 = to_tf32(A[g * lda + kk + t + 4]), a3 = to_tf32(A[(g + 8) * lda + kk + t + 4]);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const uint32_t b0 = to_tf32(B[(kk + t) * ldb + 8 * nt + g]);
-      const uint32_t b1 = to_tf32(B[(kk + t + 4) * ldb + 8 * nt + g]);
-      mma_tf32_16x8x8(acc[nt], a0, a1, a2, a3, b0, b1);
-    }
-  }
-}
-// stores s * acc (accumulator layout) as a 16 x 16 block with row stride ld
-__device__ __forceinline__ void block_store16(float *C, int ld, const float (&acc)[2][4], float s,
-                                              int lane) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    C[g * ld + 8 * nt + 2 * t] = s * acc[nt][0];
-    C[g * ld + 8 * nt + 2 * t + 1] = s * acc[nt][1];
-    C[(g + 8) * ld + 8 * nt + 2 * t] = s * acc[nt][2];
-    C[(g + 8) * ld + 8 * nt + 2 * t + 1] = s * acc[nt][3];
-  }
-}
-
 __device__ __forceinline__ uint4 pack8(const float *f) {
   uint4 v;
   v.x = pack_bf16x2(f[0], f[1]);
@@ -261,18 +195,6 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
   v.w = pack_bf16x2(f[6], f[7]);
   return v;
 }
-
-// e4m3 inputs (F8): a chunk's K, Q and V arrive as e4m3 codes (64 rows of 128
-// bytes each) in one staging buffer that aliases the fp32 A / T area, and are
-// converted to bf16 (exactly: every e4m3 value is a bf16 value) into the same
-// swizzled tiles the bf16 path loads; the next chunk's codes are loaded after
-// the current chunk's solve has finished with A and T.  The descale factors
-// fold into products the kernel forms anyway: A and (M o QK^T) take sk^2 and
-// sq sk, T' (for W) sk, T'' (for U) sv, Delta' (state update) sk, and the
-// output's Q S0^T term sq -- so no extra rounding is added.
-constexpr int SM_STAGE8 = SM_A;  // e4m3 staging: K rows at +0, Q at +8192, V at +16384
-static_assert(SM_STAGE8 % 1024 == 0 && SM_STAGE8 + 3 * 8192 <= SM_X,
-              "e4m3 staging must be 1024-aligned and end before the block-product area");
 
 // 16 e4m3 codes (one 16-byte chunk) to 16 floats, exactly
 __device__ __forceinline__ void decode16_e4m3(uint4 raw, float (&f)[16]) {
@@ -287,539 +209,6 @@ __device__ __forceinline__ void decode16_e4m3(uint4 raw, float (&f)[16]) {
       f[4 * i + 2 * h2] = f2.x;
       f[4 * i + 2 * h2 + 1] = f2.y;
     }
-  }
-}
-
-template <bool F8>
-__global__ void __launch_bounds__(kThreads, 1)
-gdn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const GdnTcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const uint32_t sb = smem_u32(smem);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int lg = warp & 3, wg = warp >> 2;  // TMEM lane group; column half
-  const int row = lg * 32 + lane;           // this thread's TMEM lane = tile row
-  const flide_tree_index &x = p.x;
-  const float dsq = F8 ? p.descale[0] : 1.f, dsk = F8 ? p.descale[1] : 1.f,
-              dsv = F8 ? p.descale[2] : 1.f;
-  float *sbeta = reinterpret_cast<float *>(smem + SM_SCAL);
-  float *sG = sbeta + C;
-  float *sgam = sG + C;
-  int *sseg = reinterpret_cast<int *>(sgam + C);
-  float *sG2 = reinterpret_cast<float *>(sseg + C);  // G * log2(e)
-  float *Am = reinterpret_cast<float *>(smem + SM_A);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
-  int *abort_flag = reinterpret_cast<int *>(smem + SM_MISC + 4);
-  auto bar = [&](int i) -> uint32_t { return sb + SM_BAR + 8 * i; };
-
-  if (tid == 0) {
-    for (int i = 0; i < NUM_BARS; ++i) mbar_init(bar(i), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncwarp();
-  if (warp == 0) {
-    tmem_alloc(sb + SM_MISC, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tl = tmem + ((uint32_t)(lg * 32) << 16);  // this warp's TMEM lanes
-  volatile int *vabort = abort_flag;
-
-  const int n_groups = failed(x.status) ? 0 : *groups_n(x, p.goff);
-  const int L0 = x.level_ptr[p.level];
-  const long items = (long)n_groups * p.H;
-  uint32_t full_phase0 = 0, full_phase1 = 0, mma_phase = 0;
-  bool pending0 = false, pending1 = false;  // loads in flight (thread 0)
-  int stage = 0;
-  bool ok = true;
-
-  auto mma_sync = [&]() -> bool {  // commit all issued MMAs and wait (every thread)
-    tc_fence_before();
-    if (tid == 0) mma_commit(bar(B_MMA));
-    __syncwarp();
-    const bool r = mbar_wait(bar(B_MMA), mma_phase, vabort, kTimeoutNs);
-    mma_phase ^= 1;
-    tc_fence_after();
-    return __syncthreads_and(r);
-  };
-
-  int *s_item = reinterpret_cast<int *>(smem + SM_MISC + 8);
-  for (;;) {
-    // next (group, head) item from the level's shared counter
-    if (tid == 0) *s_item = atomicAdd(groups_next(x, p.goff), 1);
-    __syncthreads();
-    const long it = *s_item;
-    __syncthreads();
-    if (!ok || it >= items) break;
-    const int rk = (int)(it / p.H), h = (int)(it % p.H);
-    const int grp = groups_order(x, p.goff)[rk];
-    if (grp < 0 || grp >= n_groups) {
-      if (tid == 0) check_fail(x, 6, grp);
-      break;
-    }
-    const int k0 = groups_start(x, p.goff)[grp], cnt = groups_count(x, p.goff)[grp];
-    const int Nact = x.counts[FLIDE_CNT_N], Tact = x.counts[FLIDE_CNT_T];
-    if (k0 < 0 || cnt < 1 || L0 + k0 + cnt > Nact) {
-      if (tid == 0) check_fail(x, 1, k0 * 100000L + cnt);
-      break;
-    }
-    const int n0 = x.level_node[L0 + k0];
-    const int n1 = x.level_node[L0 + k0 + cnt - 1];
-    if (n0 < 0 || n1 < n0 || n1 >= Nact) {
-      if (tid == 0) check_fail(x, 2, n0 * 100000L + n1);
-      break;
-    }
-    const int tbeg = x.node_start[n0], tend = x.node_start[n1 + 1];
-    if (tbeg < 0 || tend < tbeg || tend > Tact) {
-      if (tid == 0) check_fail(x, 3, tend);
-      break;
-    }
-    const bool scan = cnt == 1;  // single node: chunks in order, state carried
-    const int slot = x.state_slot[n0];
-    const int r = x.node_req[n0];
-    if (r < 0 || r >= x.R || (slot >= 0 && slot >= p.n_slots)) {
-      if (tid == 0) check_fail(x, 4, r * 100000L + slot);
-      break;
-    }
-    const int nchunks = (tend - tbeg + C - 1) / C;
-
-    // ---- starting state into TMEM (lane c = state row c)
-    const float *src = nullptr;
-    if (p.level == 0) {
-      if (p.state_in) src = p.state_in + ((size_t)r * p.H + h) * D * D;
-    } else {
-      const int pa = x.anc_ptr[n0 + 1] - 2;
-      const int ps = (pa >= 0 && x.depth[n0] >= 1) ? x.state_slot[x.anc_node[pa]] : -1;
-      if (ps < 0 || ps >= p.n_slots) {
-        if (tid == 0) check_fail(x, 5, ps);
-        break;
-      }
-      src = p.node_state + ((size_t)ps * p.H + h) * D * D;
-    }
-    {
-      uint32_t v[64];
-#pragma unroll
-      for (int i = 0; i < 64; i += 4) {
-        const float4 f4 = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * D + wg * 64 + i)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-        v[i] = __float_as_uint(f4.x);
-        v[i + 1] = __float_as_uint(f4.y);
-        v[i + 2] = __float_as_uint(f4.z);
-        v[i + 3] = __float_as_uint(f4.w);
-      }
-      tmem_st64(tl + R_S + wg * 64, v);
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // K, Q, V of chunk c into stage st (thread 0)
-    auto issue_loads = [&](int c, int st) {
-      const int row = tbeg + c * C;
-      if (F8) {  // codes into the one staging buffer
-        const uint32_t sg = sb + SM_STAGE8, fb = bar(B_FULL + 0);
-        pending0 = true;
-        mbar_arrive_expect_tx(fb, 3 * 8192);
-        tma_load_3d(sg, &tm_k, fb, 0, h, row);
-        tma_load_3d(sg + 8192, &tm_q, fb, 0, h, row);
-        tma_load_3d(sg + 16384, &tm_v, fb, 0, h, row);
-        return;
-      }
-      const uint32_t kq = sb + SM_KQ + st * 32768, vv = sb + SM_V + st * 16384;
-      const uint32_t fb = bar(B_FULL + st);
-      if (st == 0) pending0 = true; else pending1 = true;
-      mbar_arrive_expect_tx(fb, 6 * 8192);
-      tma_load_3d(kq, &tm_k, fb, 0, h, row);
-      tma_load_3d(kq + 16384, &tm_k, fb, 64, h, row);
-      tma_load_3d(kq + 8192, &tm_q, fb, 0, h, row);
-      tma_load_3d(kq + 16384 + 8192, &tm_q, fb, 64, h, row);
-      tma_load_3d(vv, &tm_v, fb, 0, h, row);
-      tma_load_3d(vv + 8192, &tm_v, fb, 64, h, row);
-    };
-    if (tid == 0) issue_loads(0, stage);
-    __syncwarp();
-    // per-token scalars (beta, g, node) of the next chunk, loaded into
-    // registers one chunk ahead so their latency overlaps the current chunk
-    float nb = 0.f, ng = 0.f;
-    int nn = -1;
-    auto load_scalars = [&](int c) {
-      const int t = tbeg + c * C + tid;
-      const bool v = tid < C && t < tend && t < Tact;
-      nb = v ? p.beta[(size_t)t * p.H + h] : 0.f;
-      ng = v ? p.g[(size_t)t * p.H + h] : 0.f;
-      nn = v ? x.token_node[t] - n0 : -1;
-    };
-    load_scalars(0);
-
-    for (int c = 0; ok && c < nchunks; ++c) {
-      const int st = stage;
-      const int cbeg = tbeg + c * C;
-      const int n = min(C, tend - cbeg);
-      const bool update = scan && (c + 1 < nchunks || slot >= 0);
-      const uint32_t kq = sb + SM_KQ + st * 32768, vv = sb + SM_V + st * 16384;
-      // prefetch the next chunk into the other stage (its last readers are
-      // done); e4m3 codes wait until this chunk's solve has freed the staging
-      if (!F8 && tid == 0 && c + 1 < nchunks) issue_loads(c + 1, st ^ 1);
-      __syncwarp();
-
-      // ---- per-token scalars: beta, segment id, then the segmented log decay
-      if (tid < C) {
-        sbeta[tid] = nb;
-        sG[tid] = ng;
-        sseg[tid] = nn;
-      }
-      if (c + 1 < nchunks) load_scalars(c + 1);
-      __syncthreads();
-      if (warp == 0) {
-        // segmented inclusive scan of g, two tokens per lane: (value,
-        // segment-start flag) pairs combined Hillis-Steele style
-        const int lane = tid;
-        const float a0 = sG[2 * lane], a1 = sG[2 * lane + 1];
-        const int s0 = sseg[2 * lane], s1 = sseg[2 * lane + 1];
-        const int prev_s1 = __shfl_up_sync(0xffffffffu, s1, 1);
-        const bool cont0 = lane > 0 && prev_s1 == s0;  // token 2l continues token 2l-1
-        float v = (s1 == s0) ? a0 + a1 : a1;
-        int f = (s1 != s0 || !cont0) ? 1 : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float pv = __shfl_up_sync(0xffffffffu, v, o);
-          const int pf = __shfl_up_sync(0xffffffffu, f, o);
-          if (lane >= o) {
-            if (!f) v += pv;
-            f |= pf;
-          }
-        }
-        const float carry = __shfl_up_sync(0xffffffffu, v, 1);
-        const float g0 = a0 + (cont0 ? carry : 0.f);
-        const float g1 = (s1 == s0) ? g0 + a1 : a1;
-        sG[2 * lane] = g0;
-        sG[2 * lane + 1] = g1;
-        sgam[2 * lane] = expf(g0);
-        sgam[2 * lane + 1] = expf(g1);
-        sG2[2 * lane] = g0 * 1.4426950408889634f;
-        sG2[2 * lane + 1] = g1 * 1.4426950408889634f;
-      }
-      // ---- wait for this chunk's K, Q, V
-      const int fbi = F8 ? 0 : st;
-      const bool loaded = mbar_wait(bar(B_FULL + fbi), fbi == 0 ? full_phase0 : full_phase1, vabort,
-                                    kTimeoutNs);
-      if (loaded) {
-        if (fbi == 0) { full_phase0 ^= 1; pending0 = false; }
-        else { full_phase1 ^= 1; pending1 = false; }
-      }
-      if (!__syncthreads_and(loaded)) { ok = false; break; }
-      if (F8) {
-        // e4m3 codes -> bf16 tiles of stage st: staging row rr (K 0-63, Q
-        // 64-127, V 128-191), 16-code chunk j = dims 16j .. 16j+15
-        const uint8_t *stg = smem + SM_STAGE8;
-        for (int e = tid; e < 3 * C * 8; e += kThreads) {
-          const int rr = e >> 3, j = e & 7;
-          const uint4 raw = *reinterpret_cast<const uint4 *>(stg + rr * 128 + ((j ^ (rr & 7)) << 4));
-          float f[16];
-          decode16_e4m3(raw, f);
-          const int which = rr >> 6, t = rr & (C - 1), slab = j >> 2, cc = (j & 3) * 2;
-          uint8_t *dst = which < 2 ? smem + SM_KQ + st * 32768 + slab * 16384
-                                   : smem + SM_V + st * 16384 + slab * 8192;
-          const int R = which == 1 ? t + C : t;
-          st_chunk(dst, R, cc, pack8(f));
-          st_chunk(dst, R, cc + 1, pack8(f + 8));
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-      }
-      const float gam_last = sgam[n - 1];
-
-      // ---- R1 = [K;Q] [K;Q]^T
-      if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 128, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16(tmem + R1, sdesc_sw128(kq + o, 16, 1024), sdesc_sw128(kq + o, 16, 1024), id,
-                   kk > 0 ? 1u : 0u);
-        }
-      }
-      __syncwarp();
-      // ---- meanwhile: bf16 copy of S0 (B operand, rows = dv); rescale S
-      {
-        uint32_t sr[64];
-        tmem_ld64(tl + R_S + wg * 64, sr);
-        uint8_t *s0 = smem + SM_S0 + wg * 16384;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float f[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(sr[8 * q + u]);
-          st_chunk(s0, row, q, pack8(f));
-        }
-        if (update) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) sr[i] = __float_as_uint(__uint_as_float(sr[i]) * gam_last);
-          tmem_st64(tl + R_S + wg * 64, sr);
-        }
-      }
-      if (!mma_sync()) { ok = false; break; }
-
-      // ---- A (rows 0-63 of R1) and the decayed causal QK^T (rows 64-127):
-      //      entry (i, j) scaled by gamma_i / gamma_j = 2^(G2_i - G2_j) where
-      //      j precedes (A) or equals (QK^T) i inside i's segment
-      {
-        uint32_t d1[32];  // this warp's half of the row: j = 32 wg + u
-        tmem_ld32(tl + R1 + 32 * wg, d1);
-        const int i = row & (C - 1);
-        const bool is_a = row < C;
-        const float G2i = sG2[i], scale_i = is_a ? sbeta[i] * (dsk * dsk) : dsq * dsk;
-        const int si = sseg[i];
-        const int jmax = is_a ? i - 1 : i;  // last visible j
-        const float4 *g4 = reinterpret_cast<const float4 *>(sG2);
-        const int4 *s4 = reinterpret_cast<const int4 *>(sseg);
-        float e[32];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 gv = g4[8 * wg + q];
-          const int4 sv = s4[8 * wg + q];
-          const float gj[4] = {gv.x, gv.y, gv.z, gv.w};
-          const int sj[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int jj = 4 * q + u, j = 32 * wg + jj;
-            const bool m = j <= jmax && sj[u] == si && si >= 0;
-            e[jj] = m ? scale_i * ex2_approx(G2i - gj[u]) * __uint_as_float(d1[jj]) : 0.f;
-          }
-        }
-        if (is_a) {
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) Am[i * A_LD + 32 * wg + jj] = e[jj];
-        } else {
-          uint8_t *pm = smem + SM_PM;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) st_chunk(pm, row, 4 * wg + q, pack8(e + 8 * q));  // token row i at tile row 64 + i
-        }
-      }
-      __syncthreads();
-
-      // ---- T = (I + A)^-1 by 16 x 16 blocks (A strictly lower triangular)
-      {
-        float *Tm = reinterpret_cast<float *>(smem + SM_T);
-        float *Xm = reinterpret_cast<float *>(smem + SM_X);
-        // diagonal blocks: thread (block kb, column cc), substitution down the column
-        if (tid < C) {
-          const int r0 = 16 * (tid >> 4), cc = tid & 15;
-          float tcol[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float s0 = 0.f, s1 = 0.f;
-            const float *arow = Am + (r0 + i) * A_LD + r0;
-#pragma unroll
-            for (int j = 0; j + 1 < i; j += 2) {
-              s0 = fmaf(arow[j], tcol[j], s0);
-              s1 = fmaf(arow[j + 1], tcol[j + 1], s1);
-            }
-            if (i & 1) s0 = fmaf(arow[i - 1], tcol[i - 1], s0);
-            tcol[i] = (i == cc) ? 1.f : (i > cc ? -(s0 + s1) : 0.f);
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) Tm[(r0 + i) * A_LD + r0 + cc] = tcol[i];
-        }
-        __syncthreads();
-        // block row bi: X_bj = sum_{k=j}^{bi-1} A_bk T_kj, then T_bj = -T_bb X_bj
-        // (T_bb is exactly zero above its diagonal), one warp per column block
-        // j < bi, the 16 x 16 products on the warp's tensor path; X goes
-        // through the warp's scratch block to change fragment layout
-        // T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles, one
-        // 16-row block row at a time (64 items: row, quarter of the columns):
-        // block row b - 1 is converted by two otherwise idle warps while
-        // block row b is solved
-        auto convert_block_row = [&](int b, int item) {
-          const int i = 16 * b + (item >> 2), qq = item & 3;
-          uint8_t *t1 = smem + SM_TA, *t2 = smem + SM_TA + 16384;
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            float f1[8], f2[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int j = 16 * qq + 8 * q + u;
-              const float tv = (j >> 4) <= (i >> 4) ? Tm[i * A_LD + j] : 0.f;
-              f1[u] = F8 ? tv * (sbeta[j] * sgam[j] * dsk) : tv * sbeta[j] * sgam[j];
-              f2[u] = F8 ? tv * (sbeta[j] * dsv) : tv * sbeta[j];
-            }
-            st_chunk(t1, i, 2 * qq + q, pack8(f1));
-            st_chunk(t2, i, 2 * qq + q, pack8(f2));
-          }
-        };
-        for (int bi = 1; bi < 4; ++bi) {
-          if (warp >= 3 && warp < 5) convert_block_row(bi - 1, tid - 96);
-          if (warp < bi) {
-            const int j = warp;
-            float acc[2][4] = {};
-            for (int k = j; k < bi; ++k)
-              block_mma16(acc, Am + 16 * bi * A_LD + 16 * k, A_LD, Tm + 16 * k * A_LD + 16 * j, A_LD, lane);
-            float *xs = Xm + j * 16 * X_LD;
-            block_store16(xs, X_LD, acc, 1.f, lane);
-            __syncwarp();
-            float acc2[2][4] = {};
-            block_mma16(acc2, Tm + 16 * bi * A_LD + 16 * bi, A_LD, xs, X_LD, lane);
-            block_store16(Tm + 16 * bi * A_LD + 16 * j, A_LD, acc2, -1.f, lane);
-          }
-          __syncthreads();
-        }
-        if (tid < 64) convert_block_row(3, tid);
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      // the staging area (A, T) is free now: the next chunk's e4m3 codes
-      if (F8 && tid == 0 && c + 1 < nchunks) issue_loads(c + 1, 0);
-
-      // ---- R2 = T' K (= W),  R3 = T'' V (= U)
-      if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 128, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16(tmem + R2, sdesc_sw128(sb + SM_TA + kk * 32, 16, 1024),
-                   sdesc_sw128(kq + kk * 2048, 16384, 1024), id, kk > 0 ? 1u : 0u);
-          mma_bf16(tmem + R3, sdesc_sw128(sb + SM_TA + 16384 + kk * 32, 16, 1024),
-                   sdesc_sw128(vv + kk * 2048, 8192, 1024), id, kk > 0 ? 1u : 0u);
-        }
-      }
-      if (!mma_sync()) { ok = false; break; }
-
-      // ---- -W (token rows) as a K-major A operand over T' / T''
-      if (row < C) {
-        uint32_t w[64];
-        tmem_ld64(tl + R2 + wg * 64, w);
-        uint8_t *nw = smem + SM_TA + wg * 16384;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float f[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) f[u] = -__uint_as_float(w[8 * q + u]);
-          st_chunk(nw, row, q, pack8(f));
-        }
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-
-      // ---- R3 += (-W) S0^T (= Delta);  R1 = [K;Q] S0^T (rows 64-127: Q S0^T)
-      if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 128, false);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t b = sdesc_sw128(sb + SM_S0 + o, 16, 1024);
-          mma_bf16(tmem + R3, sdesc_sw128(sb + SM_TA + o, 16, 1024), b, id, 1u);
-          mma_bf16(tmem + R1, sdesc_sw128(kq + o, 16, 1024), b, id, kk > 0 ? 1u : 0u);
-        }
-      }
-      if (!mma_sync()) { ok = false; break; }
-
-      // ---- Delta rows (token j) -> MN-major B over S0's first half, and
-      //      Delta'^T = (Delta * gamma_last/gamma_j)^T -> K-major A (second half)
-      if (row < C) {
-        const int j = row;  // token; this warp handles dv = 64 wg .. 64 wg + 63
-        uint32_t dr[64];
-        tmem_ld64(tl + R3 + wg * 64, dr);
-        uint8_t *db = smem + SM_S0 + wg * 8192;
-        __nv_bfloat16 *dat = reinterpret_cast<__nv_bfloat16 *>(smem + SM_S0 + 16384);
-        const float sc = F8 ? gam_last / sgam[j] * dsk : gam_last / sgam[j];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float f[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(dr[8 * q + u]);
-          st_chunk(db, j, q, pack8(f));
-        }
-        if (update) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            dat[sw_elem(64 * wg + c, j) >> 1] = __float2bfloat16_rn(__uint_as_float(dr[c]) * sc);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-
-      // ---- R2 = (M o QK^T) Delta (rows 64-127);  S += Delta'^T K
-      if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_bf16(128, 128, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16(tmem + R2, sdesc_sw128(sb + SM_PM + kk * 32, 16, 1024),
-                   sdesc_sw128(sb + SM_S0 + kk * 2048, 8192, 1024), id, kk > 0 ? 1u : 0u);
-          if (update)
-            mma_bf16(tmem + R_S, sdesc_sw128(sb + SM_S0 + 16384 + kk * 32, 16, 1024),
-                     sdesc_sw128(kq + kk * 2048, 16384, 1024), id, 1u);
-        }
-      }
-      if (!mma_sync()) { ok = false; break; }
-
-      // ---- outputs (token rows 64-127): o_i = gamma_i (Q S0^T)_i + ((M o QK^T) Delta)_i
-      if (row >= C) {
-        const int i = row - C;
-        const bool valid = i < n && cbeg + i < Tact;
-        __nv_bfloat16 *o = p.out + ((size_t)(cbeg + i) * p.H + h) * D;
-        const float gi = F8 ? sgam[i] * dsq : sgam[i];
-        {
-          const int half = wg;  // this warp's 64 output dims
-          uint32_t o1[32], o2[32];
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            tmem_ld32(tl + R1 + half * 64 + qq * 32, o1);
-            tmem_ld32(tl + R2 + half * 64 + qq * 32, o2);
-            if (valid) {
-#pragma unroll
-              for (int q8 = 0; q8 < 4; ++q8) {
-                float f[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                  f[u] = fmaf(gi, __uint_as_float(o1[q8 * 8 + u]), __uint_as_float(o2[q8 * 8 + u]));
-                *reinterpret_cast<uint4 *>(o + half * 64 + qq * 32 + q8 * 8) = pack8(f);
-              }
-            }
-          }
-        }
-      }
-      stage ^= 1;
-      __syncthreads();
-    }
-    if (!ok) break;
-
-    // ---- end state of a node with a slot
-    if (scan && slot >= 0) {
-      uint32_t sr[64];
-      tmem_ld64(tl + R_S + wg * 64, sr);
-      float *dst = p.node_state + ((size_t)slot * p.H + h) * D * D + (size_t)row * D + wg * 64;
-#pragma unroll
-      for (int i = 0; i < 64; i += 4)
-        *reinterpret_cast<float4 *>(dst + i) =
-            make_float4(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1]),
-                        __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
-    }
-    __syncthreads();
-  }
-
-  if (!ok) {
-    // drain: loads this CTA may still have in flight, and its MMAs
-    if (tid == 0) {
-      if (pending0) mbar_wait(bar(B_FULL + 0), full_phase0, vabort, kTimeoutNs, false);
-      if (pending1) mbar_wait(bar(B_FULL + 1), full_phase1, vabort, kTimeoutNs, false);
-      mma_commit(bar(B_MMA));
-      mbar_wait(bar(B_MMA), mma_phase, vabort, kTimeoutNs, false);
-      set_status(x.status, FLIDE_ERR_TIMEOUT);
-    }
-  }
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1062,9 +451,14 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!wait_w(bar(V_EMPTY), (pv_seq & 1) ^ 1)) return false;
       if (lane == 0) {
         const uint32_t vb = sb + V, fb = bar(V_FULL);
-        mbar_arrive_expect_tx(fb, 16384);
-        tma_load_3d(vb, &tm_v, fb, 0, pv_h, pv_cbeg);
-        tma_load_3d(vb + 8192, &tm_v, fb, 64, pv_h, pv_cbeg);
+        if (F8) {
+          mbar_arrive_expect_tx(fb, 8192);
+          tma_load_3d(vb + 8192, &tm_v, fb, 0, pv_h, pv_cbeg);
+        } else {
+          mbar_arrive_expect_tx(fb, 16384);
+          tma_load_3d(vb, &tm_v, fb, 0, pv_h, pv_cbeg);
+          tma_load_3d(vb + 8192, &tm_v, fb, 64, pv_h, pv_cbeg);
+        }
       }
       last_v = (int)pv_seq;
       pend_v = false;
@@ -1178,11 +572,17 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!wait_w(bar(KQ_EMPTY + s), ((seq >> 1) & 1) ^ 1)) { ok = false; break; }
         if (lane == 0) {
           const uint32_t kq = sb + KQ + s * 32768, fb = bar(KQ_FULL + s);
-          mbar_arrive_expect_tx(fb, 32768);
-          tma_load_3d(kq, &tm_q, fb, 0, h, cbeg);
-          tma_load_3d(kq + 16384, &tm_q, fb, 64, h, cbeg);
-          tma_load_3d(kq + 8192, &tm_k, fb, 0, h, cbeg);
-          tma_load_3d(kq + 16384 + 8192, &tm_k, fb, 64, h, cbeg);
+          if (F8) {  // e4m3 codes (one 128-byte row per token) into the second slabs
+            mbar_arrive_expect_tx(fb, 16384);
+            tma_load_3d(kq + 16384, &tm_q, fb, 0, h, cbeg);
+            tma_load_3d(kq + 16384 + 8192, &tm_k, fb, 0, h, cbeg);
+          } else {
+            mbar_arrive_expect_tx(fb, 32768);
+            tma_load_3d(kq, &tm_q, fb, 0, h, cbeg);
+            tma_load_3d(kq + 16384, &tm_q, fb, 64, h, cbeg);
+            tma_load_3d(kq + 8192, &tm_k, fb, 0, h, cbeg);
+            tma_load_3d(kq + 16384 + 8192, &tm_k, fb, 64, h, cbeg);
+          }
         }
         last_kq[s] = (int)(seq >> 1);
         // the previous chunk's V: its buffer frees when that chunk's prep
@@ -1221,6 +621,32 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (pt == 0) r = mbar_wait(b, parity, vabort, kTimeoutNs);
       return role_and(BAR_PREP, NP, r);
     };
+    // e4m3 codes (one swizzled 128-byte row per token, staged in the second
+    // slab) -> the bf16 tiles: dims 0-63 to the first slab, dims 64-127 over
+    // the codes themselves, so every code is read before any is overwritten.
+    // Exact: every e4m3 value is a bf16 value.  base = first slab, ss = slab
+    // stride, tiles = 8 KB tiles per slab (tile t at +8192 t).
+    auto expand_e4m3 = [&](uint8_t *base, int ss, int tiles) {
+      uint4 raw[4];
+      const int per = tiles * C * 8 / NP;  // 16-byte code chunks per thread (2 or 4)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (u >= per) break;
+        const int e = pt + NP * u, tt = e >> 9, r = (e >> 3) & (C - 1), j = e & 7;
+        raw[u] = *reinterpret_cast<const uint4 *>(base + ss + tt * 8192 + r * 128 + ((j ^ (r & 7)) << 4));
+      }
+      role_sync(BAR_PREP, NP);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (u >= per) break;
+        const int e = pt + NP * u, tt = e >> 9, r = (e >> 3) & (C - 1), j = e & 7;
+        float f[16];
+        decode16_e4m3(raw[u], f);
+        uint8_t *dst = base + (j >> 2) * ss + tt * 8192;
+        st_chunk(dst, r, 2 * (j & 3), pack8(f));
+        st_chunk(dst, r, 2 * (j & 3) + 1, pack8(f + 8));
+      }
+    };
     // A chunk's start: its job, its Q and K (rows past its tokens zeroed:
     // they may hold another node's tokens or uninitialised memory) and its
     // [Q;K][Q;K]^T into G.  1 = the producer's stop job, -1 = a wait gave up.
@@ -1231,6 +657,10 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int nn = jn->n, ss = sq & 1;
       uint8_t *kqn = smem + KQ + ss * 32768;
       if (!wait_r(bar(KQ_FULL + ss), (sq >> 1) & 1)) return -1;
+      if (F8) {
+        expand_e4m3(kqn, 16384, 2);
+        if (nn < C) role_sync(BAR_PREP, NP);  // the zeroing below rewrites expanded rows
+      }
       if (nn < C) {
         for (int e = pt; e < 4 * C * 8; e += NP) {  // (slab, Q|K, row, 16-byte chunk)
           const int r = (e >> 3) & (C - 1);
@@ -1238,6 +668,8 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             *reinterpret_cast<uint4 *>(kqn + (e >> 10) * 16384 + ((e >> 9) & 1) * 8192 + r * 128 +
                                        (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
+      }
+      if (F8 || nn < C) {
         fence_proxy_async_smem();
         role_sync(BAR_PREP, NP);
       }
@@ -1409,6 +841,10 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // -- 6. V (rows past the chunk zeroed), then W = T' K -> W and
       //       U = [T''; 0] V -> X once the epilogue of chunk seq-1 has read X
       if (!wait_r(bar(V_FULL), seq & 1)) break;
+      if (F8) {
+        expand_e4m3(smem + V, 8192, 1);
+        if (n < C) role_sync(BAR_PREP, NP);  // the zeroing below rewrites expanded rows
+      }
       if (n < C) {
         for (int e = pt; e < 2 * C * 8; e += NP) {
           const int r = (e >> 3) & (C - 1);
@@ -1739,7 +1175,8 @@ int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, con
   if (cudaGetDevice(&dev) != cudaSuccess) return FLIDE_ERR_CUDA;
   if (dev < 0 || dev >= 64 || !attr_set[f8][dev].load(std::memory_order_acquire)) {
     const cudaError_t e =
-        f8 ? cudaFuncSetAttribute(gdn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
+        f8 ? cudaFuncSetAttribute(gdn_ws_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ws::SMEM_BYTES)
            : cudaFuncSetAttribute(gdn_ws_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   ws::SMEM_BYTES);
     if (e != cudaSuccess) return FLIDE_ERR_CUDA;
@@ -1763,7 +1200,7 @@ int fork_gdn_tc(const void *q, const void *k, const void *v, const float *g, con
     gdn_groups_kernel<<<1, 1024, 0, s>>>(*x, lvl, prm.goff);
     FLIDE_LAUNCH_CHECK();
     if (f8)
-      gdn_tc_kernel<true><<<sms, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, prm);
+      gdn_ws_kernel<true><<<sms, ws::kThreads, ws::SMEM_BYTES, s>>>(mq, mk, mv, prm);
     else
       gdn_ws_kernel<false><<<sms, ws::kThreads, ws::SMEM_BYTES, s>>>(mq, mk, mv, prm);
     FLIDE_LAUNCH_CHECK();
