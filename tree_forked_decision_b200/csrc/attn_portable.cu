@@ -78,7 +78,12 @@ attn_portable_kernel(PortableArgs<T> a) {
   for (long row = (long)blockIdx.x * kWarps + warp; row < rows; row += (long)gridDim.x * kWarps) {
     const int t = (int)(row / a.Hq), h = (int)(row % a.Hq);
     const int kvh = h / G;
+    const int Nact = x.counts[FLIDE_CNT_N];
+    // debug build: the token's node and request index the tree arrays
     const int n = x.token_node[t];
+    if (!in_bounds(x.status, x.counts, n, Nact, 301) ||
+        !in_bounds(x.status, x.counts, x.node_req[n], x.R, 302))
+      continue;
     const int r = x.node_req[n];
     __syncwarp();
     for (int c = lane; c < a.d; c += 32)
@@ -104,7 +109,8 @@ attn_portable_kernel(PortableArgs<T> a) {
     // 2. strict ancestors, root first
     const int a0 = x.anc_ptr[n], a1 = x.anc_ptr[n + 1] - 1;
     for (int i = a0; i < a1; ++i) {
-      const int an = x.anc_node[i];
+      const int an = x.anc_node[checked(x.status, x.counts, i, (long long)x.N * (x.max_depth + 1), 303)];
+      if (!in_bounds(x.status, x.counts, an, Nact, 304)) continue;
       const int s0 = x.node_start[an], sl = x.node_start[an + 1] - s0;
       if (sl > 0) attend_span(a, a.k, a.v, s0, sl, kvh, qs, m, l, acc);
     }

@@ -199,6 +199,8 @@ branch_logprob_kernel(const __grid_constant__ CUtensorMap tm_h,
       const uint32_t tl = tmem + ((uint32_t)(lg * 32) << 16);
       const bool real = row < nrows;
       const int y = real ? p.targets[row0 + row] : -1;
+      // debug build: a target outside the vocabulary would score no logit
+      if (real) in_bounds(p.x.status, p.x.counts, y, p.V, 601);
       float m2 = -INFINITY, s = 0.f, tgt = -INFINITY;  // running max (log2 units), sum, target logit
       bool ok = true;
       for (int v = v0; v < v1; ++v) {

@@ -58,6 +58,11 @@ gdn_level_kernel(GdnArgs<T> a) {
     const int blk = (int)(it % nblk);
     const int h = (int)((it / nblk) % a.H);
     const int n = x.level_node[l0 + (int)(it / ((long)nblk * a.H))];
+    // debug build: node, request and parent index the tree arrays (the whole
+    // block takes the same branch: one item per block)
+    if (!in_bounds(x.status, x.counts, n, x.counts[FLIDE_CNT_N], 321) ||
+        !in_bounds(x.status, x.counts, x.node_req[n], x.R, 322))
+      return;
     const int r = x.node_req[n];
     const int vrow = blk * kRows + row;
 
@@ -68,6 +73,7 @@ gdn_level_kernel(GdnArgs<T> a) {
       if (a.state_in) src = a.state_in + ((size_t)r * a.H + h) * SS;
     } else {
       const int pg = x.anc_node[x.anc_ptr[n + 1] - 2];  // parent (global id)
+      if (!in_bounds(x.status, x.counts, pg, x.counts[FLIDE_CNT_N], 323)) return;
       const int ps = x.state_slot[pg];
       if (ps < 0 || ps >= a.n_slots) { set_status(x.status, FLIDE_ERR_CAPACITY); return; }
       src = a.node_state + ((size_t)ps * a.H + h) * SS;
@@ -80,6 +86,9 @@ gdn_level_kernel(GdnArgs<T> a) {
     }
 
     const int t0 = x.node_start[n], t1 = x.node_start[n + 1];
+    if (!in_bounds(x.status, x.counts, t0, x.counts[FLIDE_CNT_T] + 1, 324) ||
+        !in_bounds(x.status, x.counts, t1, x.counts[FLIDE_CNT_T] + 1, 324))
+      return;
     for (int tb = t0; tb < t1; tb += TC) {
       const int cnt = min(TC, t1 - tb);
       __syncthreads();

@@ -93,6 +93,12 @@ __global__ void gdn_groups_kernel(flide_tree_index x, int level, int goff) {
   // 1: run starts
   for (int k = threadIdx.x; k < n; k += blockDim.x) {
     const int node = x.level_node[L0 + k];
+    // debug build: a level's nodes index the tree arrays
+    if (!in_bounds(x.status, x.counts, node, x.counts[FLIDE_CNT_N], 311) ||
+        (k > 0 && !in_bounds(x.status, x.counts, x.level_node[L0 + k - 1], x.counts[FLIDE_CNT_N], 311))) {
+      flag[k] = 1;
+      continue;
+    }
     int f = 1;
     if (k > 0) {
       const int prev = x.level_node[L0 + k - 1];
@@ -506,7 +512,11 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (p.state_in) src = p.state_in + ((size_t)r * p.H + h) * D * D;
           } else {
             const int pa = x.anc_ptr[n0 + 1] - 2;
-            const int ps = (pa >= 0 && x.depth[n0] >= 1) ? x.state_slot[x.anc_node[pa]] : -1;
+            // debug build: the parent entry and the parent node index the tree arrays
+            const bool pok = pa >= 0 && x.depth[n0] >= 1 &&
+                             in_bounds(x.status, x.counts, pa, (long long)x.N * (x.max_depth + 1), 313) &&
+                             in_bounds(x.status, x.counts, x.anc_node[pa], Nact, 314);
+            const int ps = pok ? x.state_slot[x.anc_node[pa]] : -1;
             if (ps < 0 || ps >= p.n_slots) { site = 5; val = ps; }
             else src = p.node_state + ((size_t)ps * p.H + h) * D * D;
           }
@@ -553,6 +563,9 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float a0 = v0 ? p.g[i0] : 0.f, a1 = v1 ? p.g[i1] : 0.f;
         const int s0 = v0 ? x.token_node[cbeg + t0] - n0 : -1;
         const int s1 = v1 ? x.token_node[cbeg + t1] - n0 : -1;
+        // debug build: a token of the item belongs to one of its nodes
+        if (v0) in_bounds(x.status, x.counts, s0, cnt, 315);
+        if (v1) in_bounds(x.status, x.counts, s1, cnt, 315);
         if (lane == 0) {
           jb->stop = 0;
           jb->cbeg = cbeg;

@@ -91,13 +91,16 @@ __global__ void history_append_kernel(flide_tree_index x, const int32_t *req_slo
         if (lane == 0) set_status(x.status, FLIDE_ERR_CAPACITY);
         continue;
       }
+      // debug build: the root row lies in the stream (pool block ids come from
+      // the host allocator; their range is not passed to the device)
+      if (!in_bounds(x.status, x.counts, (long long)t0 + i, x.counts[FLIDE_CNT_T], 502)) continue;
       copy_row16(pool_k + pr * row_bytes, k + (size_t)(t0 + i) * row_bytes, row_bytes, lane);
       copy_row16(pool_v + pr * row_bytes, v + (size_t)(t0 + i) * row_bytes, row_bytes, lane);
     }
     // the root's end state becomes the request's state
     if (node_state && pool_S) {
       const int slot = x.state_slot[n0];
-      if (slot < 0) continue;
+      if (slot < 0 || !in_bounds(x.status, x.counts, slot, x.counts[FLIDE_CNT_SLOTS], 501)) continue;
       const float4 *src = reinterpret_cast<const float4 *>(node_state + (size_t)slot * state_floats);
       float4 *dst = reinterpret_cast<float4 *>(pool_S + (size_t)s * state_floats);
       for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < state_floats / 4;

@@ -46,6 +46,7 @@ __global__ void save_kv_kernel(flide_tree_index x, const char *k, const char *v,
   const int lane = threadIdx.x & 31;
   for (int i = warp; i < C; i += nwarps) {
     const int r = upper_bound_i(x.ckpt_start, R + 1, i) - 1;
+    if (!in_bounds(x.status, x.counts, r, R, 401)) continue;  // debug build
     const int o = i - x.ckpt_start[r];
     const int plen = x.past_start[r + 1] - x.past_start[r];
     const char *sk, *sv;
@@ -57,6 +58,9 @@ __global__ void save_kv_kernel(flide_tree_index x, const char *k, const char *v,
       int root = -1;
       // the request owns at least one node here (it has root rows)
       root = upper_bound_i(x.node_req, x.counts[FLIDE_CNT_N], r - 1);
+      if (!in_bounds(x.status, x.counts, root, x.counts[FLIDE_CNT_N], 402) ||
+          !in_bounds(x.status, x.counts, (long long)x.node_start[root] + (o - plen), x.counts[FLIDE_CNT_T], 403))
+        continue;  // debug build: the root row lies in the stream
       const size_t t = (size_t)x.node_start[root] + (o - plen);
       sk = k + t * row_bytes;
       sv = v + t * row_bytes;
@@ -82,7 +86,9 @@ __global__ void save_state_kernel(flide_tree_index x, const float *node_state, i
     float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
     if (root < N && x.node_req[root] == r) {
       const int slot = x.state_slot[root];
-      val = ((const float4 *)(node_state + (size_t)slot * H * SS))[w];
+      // debug build: the root's slot lies in the node-state buffer the tree needs
+      if (in_bounds(x.status, x.counts, slot, x.counts[FLIDE_CNT_SLOTS], 404))
+        val = ((const float4 *)(node_state + (size_t)slot * H * SS))[w];
     }
     ((float4 *)(ckpt_S + (size_t)r * H * SS))[w] = val;
   }
