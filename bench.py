@@ -314,7 +314,8 @@ def measured_peaks():
 
 
 def traffic_for(kernel_name: str, src_file: str):
-    """dram read+write bytes per launch for `kernel_name` from the committed ncu
+    """dram read+write bytes of `kernel_name` per timed unit (one launch for
+    attention, one layer = all tree levels for GDN) from the committed ncu
     summary, or None when the kernel source changed since it was captured."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -325,7 +326,7 @@ def traffic_for(kernel_name: str, src_file: str):
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     if rec.get("source_sha") != sha:
         return None
-    return rec.get("bytes_per_launch")
+    return rec.get("bytes_per_layer", rec.get("bytes_per_launch"))
 
 
 def dist_env():
@@ -750,9 +751,9 @@ def main():
         kernels["fork_gdn"] = {"ms": gdn_ms, "algorithmic_bytes": gbytes, "gbs": gdn_gbs,
                                "frac_of_hbm_peak": gdn_gbs / hbm, "bound": "hbm"}
         roofline_gdn = roofline = {
-            "kernel": "gdn_tc_kernel (GDN fork scan, tcgen05)", "bound": "hbm", "achieved": gdn_gbs,
-            "peak": hbm, "unit": "GB/s", "frac": gdn_gbs / hbm,
-            "traffic": traffic_for("gdn_tc_kernel", "gdn_tc.cu"),
+            "kernel": "gdn_ws_kernel (GDN fork scan, warp-specialised tcgen05; all tree levels)",
+            "bound": "hbm", "achieved": gdn_gbs, "peak": hbm, "unit": "GB/s", "frac": gdn_gbs / hbm,
+            "traffic": traffic_for("gdn_ws_kernel", "gdn_tc.cu"),
             "peak_source": f"{peak_src}: HBM copy bandwidth",
             "algorithmic_bytes_per_launch": gbytes, "avg_launch_ms": gdn_ms}
     if a is not None:

@@ -19,6 +19,7 @@ FANOUT = {
     "gdn_fanout_bf16": (8, 4096, 64, 16, None, (16, 128, 128), torch.bfloat16),
     "large_fanout_bf16": (4, 32768, 256, 8, (32, 8, 128), (32, 128, 128), torch.bfloat16),
     "attn_longprefix_bf16": (1, 32768, 256, 8, (4, 1, 128), None, torch.bfloat16),
+    "large_fanout_req_bf16": (1, 32768, 256, 8, (32, 8, 128), (32, 128, 128), torch.bfloat16),
 }
 
 

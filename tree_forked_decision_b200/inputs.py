@@ -295,6 +295,7 @@ WORKLOADS = {
     "mixed_hybrid_bf16": dict(idx=4, desc="32 requests depth 1-3, 2-256 options, prefix 256-8192, branches 4-64, half resumed; attn Hq=16 Hkv=4 d=128 + GDN 16x128, bf16"),
     "large_fanout_bf16": dict(idx=5, desc="4 requests, prefix 32768, 256 branches x 8, attn Hq=32 Hkv=8 d=128 + GDN 32 heads dk=dv=128, bf16"),
     "attn_longprefix_bf16": dict(idx=6, desc="1 request, prefix 32768, 256 branches x 8, GQA Hq=4 Hkv=1 d=128, bf16 (one kv group of the large fan-out request: a small case for kernel profiles)"),
+    "large_fanout_req_bf16": dict(idx=7, desc="1 request, prefix 32768, 256 branches x 8, attn Hq=32 Hkv=8 d=128 + GDN 32 heads dk=dv=128, bf16 (one request of the large fan-out batch: inputs above L2 but a quarter of the size, for DRAM-byte profiles)"),
 }
 
 
@@ -316,6 +317,9 @@ def workload(name: str, seed: int | None = None):
     if name == "attn_longprefix_bf16":
         tree = fanout_tree(1, 32768, 256, 8)
         return tree, dict(Hq=4, Hkv=1, d=128), None, torch.bfloat16, rng
+    if name == "large_fanout_req_bf16":
+        tree = fanout_tree(1, 32768, 256, 8)
+        return tree, dict(Hq=32, Hkv=8, d=128), dict(H=32, dk=128, dv=128, gate_scale=0.1), torch.bfloat16, rng
     if name == "large_fanout_bf16":
         tree = fanout_tree(4, 32768, 256, 8)
         return tree, dict(Hq=32, Hkv=8, d=128), dict(H=32, dk=128, dv=128, gate_scale=0.1), torch.bfloat16, rng
