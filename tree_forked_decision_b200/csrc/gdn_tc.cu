@@ -256,8 +256,8 @@ constexpr int CA = 98304;      // [-W; gamma Q] A tile, dk slab b at +16384 b
 constexpr int CK = 131072;     // K rows for the state update (MN-major B), dk slab b at +8192 b
 constexpr int SD = 147456;     // bf16 S0 (dk slab b at +16384 b); then Delta (+0) and Delta' (+16384)
 constexpr int TT = 180224;     // T' (+0), T'' (+8192), zeros (+16384); solve scratch during the solve
-constexpr int PM = 204800;     // fp32 [64][65]: T below the diagonal, A^T above it
-constexpr int P_LD = 65;
+constexpr int PM = 204800;     // fp32 [64][68]: T below the diagonal, A^T above it
+constexpr int P_LD = 68;       // row stride: 16-byte rows, and 8 consecutive rows on distinct banks
 constexpr int JOB = PM + C * P_LD * 4;  // 4 chunk jobs
 constexpr int JOB_BYTES = 1600;
 constexpr int BARS = JOB + 4 * JOB_BYTES;
@@ -664,12 +664,17 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // they may hold another node's tokens or uninitialised memory) and its
     // [Q;K][Q;K]^T into G.  1 = the producer's stop job, -1 = a wait gave up.
     auto start_chunk = [&](uint32_t sq) -> int {
-      if (!wait_r(bar(JOB_FULL + (sq & 3)), (sq >> 2) & 1)) return -1;
+      // the job and its [Q;K] tiles (a stop job has none), one barrier
+      bool r = true;
+      if (pt == 0) {
+        r = mbar_wait(bar(JOB_FULL + (sq & 3)), (sq >> 2) & 1, vabort, kTimeoutNs);
+        if (r && !job(sq & 3)->stop) r = mbar_wait(bar(KQ_FULL + (sq & 1)), (sq >> 1) & 1, vabort, kTimeoutNs);
+      }
+      if (!role_and(BAR_PREP, NP, r)) return -1;
       const Job *jn = job(sq & 3);
       if (jn->stop) return 1;
       const int nn = jn->n, ss = sq & 1;
       uint8_t *kqn = smem + KQ + ss * 32768;
-      if (!wait_r(bar(KQ_FULL + ss), (sq >> 1) & 1)) return -1;
       if (F8) {
         expand_e4m3(kqn, 16384, 2);
         if (nn < C) role_sync(BAR_PREP, NP);  // the zeroing below rewrites expanded rows
@@ -754,18 +759,31 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       //       then the off-diagonal blocks by doubling: T_10, T_32 from
       //       T_ii (-A_ij) T_jj, then the lower-left 32 x 32 block the same way
       if (pt < C) {
+        // column cc of the diagonal block at r0, right-looking: as soon as
+        // t_i is final every later row k takes its term -A(k, i) t_i, so one
+        // FMA per step is on the critical path.  Column i of the block's A
+        // (row r0 + i of the transposed copy) is contiguous: four 16-byte
+        // loads, issued one step ahead.
         const int r0 = 16 * (pt >> 4), cc = pt & 15;
         float tcol[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float s0 = 0.f, s1 = 0.f;
+        for (int k = 0; k < 16; ++k) tcol[k] = 0.f;
+        float4 nx[4];
 #pragma unroll
-          for (int j = 0; j + 1 < i; j += 2) {
-            s0 = fmaf(a_at(Pm, r0 + i, r0 + j), tcol[j], s0);
-            s1 = fmaf(a_at(Pm, r0 + i, r0 + j + 1), tcol[j + 1], s1);
+        for (int q = 0; q < 4; ++q) nx[q] = reinterpret_cast<const float4 *>(Pm + r0 * P_LD + r0)[q];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float col[16] = {nx[0].x, nx[0].y, nx[0].z, nx[0].w, nx[1].x, nx[1].y, nx[1].z, nx[1].w,
+                                 nx[2].x, nx[2].y, nx[2].z, nx[2].w, nx[3].x, nx[3].y, nx[3].z, nx[3].w};
+          if (i + 1 < 16) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              nx[q] = reinterpret_cast<const float4 *>(Pm + (r0 + i + 1) * P_LD + r0)[q];
           }
-          if (i & 1) s0 = fmaf(a_at(Pm, r0 + i, r0 + i - 1), tcol[i - 1], s0);
-          tcol[i] = (i == cc) ? 1.f : (i > cc ? -(s0 + s1) : 0.f);
+          const float ti = (i == cc) ? 1.f : (i > cc ? tcol[i] : 0.f);
+          tcol[i] = ti;
+#pragma unroll
+          for (int k = i + 1; k < 16; ++k) tcol[k] = fmaf(-col[k], ti, tcol[k]);
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -835,15 +853,21 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       role_sync(BAR_PREP, NP);
       // -- 5. T' = T diag(b gamma), T'' = T diag(b) as bf16 K-major A tiles
       {
-        const int i = pt >> 2, qq = pt & 3;  // row, 16-column quarter
+        // row i along the warp (8 consecutive rows fall on distinct banks),
+        // 16-column quarter qq per warp pair
+        const int i = pt & (C - 1), qq = pt >> 6;
+        const float *trow = Pm + i * P_LD + 16 * qq;
         uint8_t *t1 = smem + TT, *t2 = smem + TT + 8192;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
+          const float4 lo4 = reinterpret_cast<const float4 *>(trow + 8 * q)[0];
+          const float4 hi4 = reinterpret_cast<const float4 *>(trow + 8 * q)[1];
+          const float tr[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
           float f1[8], f2[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int j = 16 * qq + 8 * q + u;
-            const float tv = t_at(Pm, i, j), b = jb->beta[j];
+            const float tv = j < i ? tr[u] : (j == i ? 1.f : 0.f), b = jb->beta[j];
             f1[u] = tv * (b * jb->gam[j] * dsk);
             f2[u] = tv * (b * dsv);
           }
@@ -853,7 +877,16 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       // -- 6. V (rows past the chunk zeroed), then W = T' K -> W and
       //       U = [T''; 0] V -> X once the epilogue of chunk seq-1 has read X
-      if (!wait_r(bar(V_FULL), seq & 1)) break;
+      // T' and T'' are written; V has arrived and X is free (the epilogue of
+      // chunk seq-1 has read it): one barrier for the three
+      fence_proxy_async_smem();
+      {
+        bool r = true;
+        if (pt == 0)
+          r = mbar_wait(bar(V_FULL), seq & 1, vabort, kTimeoutNs) &&
+              mbar_wait(bar(XFREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
+        if (!role_and(BAR_PREP, NP, r)) break;
+      }
       if (F8) {
         expand_e4m3(smem + V, 8192, 1);
         if (n < C) role_sync(BAR_PREP, NP);  // the zeroing below rewrites expanded rows
@@ -866,8 +899,10 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();
-      if (!wait_r(bar(XFREE), (seq & 1) ^ 1)) break;
+      if (F8 || n < C) {
+        fence_proxy_async_smem();
+        role_sync(BAR_PREP, NP);
+      }
       if (pt == 0) {
         tc_fence_after();
         constexpr uint32_t id = idesc_bf16(128, 128, true);
@@ -882,18 +917,21 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mma_commit(bar(WU));
       }
       __syncwarp();
-      if (!wait_r(bar(WU), seq & 1)) break;
-      tc_fence_after();
-      if (pt == 0) mbar_arrive(bar(V_EMPTY));
-      // -- 7. the chain's tiles, once chunk seq-1's chain has finished with
-      //       them: [-W; gamma Q] (read by its first product) and K (by its
-      //       update); both are long free when the prep is the slower role
-      if (pt == 0) {
-        bool r = mbar_wait(bar(CA_FREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
-        r = r && mbar_wait(bar(CK_FREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
-        if (!r) *vabort = 1;
+      // -- 7. W and U are done (V is free again), and the chain's tiles, once
+      //       chunk seq-1's chain has finished with them: [-W; gamma Q] (read
+      //       by its first product) and K (by its update); both are long free
+      //       when the prep is the slower role.  One barrier.
+      {
+        bool r = true;
+        if (pt == 0) {
+          r = mbar_wait(bar(WU), seq & 1, vabort, kTimeoutNs);
+          if (r) mbar_arrive(bar(V_EMPTY));
+          r = r && mbar_wait(bar(CA_FREE), (seq & 1) ^ 1, vabort, kTimeoutNs) &&
+              mbar_wait(bar(CK_FREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
+        }
+        if (!role_and(BAR_PREP, NP, r)) break;
       }
-      if (!role_and(BAR_PREP, NP, *vabort == 0 || pt != 0)) break;
+      tc_fence_after();
       if (row < C) {
         // W row = token (TMEM lanes 0-63), dk half hb
         uint32_t w[64];
