@@ -878,13 +878,16 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // -- 6. V (rows past the chunk zeroed), then W = T' K -> W and
       //       U = [T''; 0] V -> X once the epilogue of chunk seq-1 has read X
       // T' and T'' are written; V has arrived and X is free (the epilogue of
-      // chunk seq-1 has read it): one barrier for the three
+      // chunk seq-1 has read it): one barrier for the three.  The e4m3 path
+      // expands V's codes first and waits for X after, so the expansion runs
+      // while the epilogue may still hold X.
       fence_proxy_async_smem();
       {
         bool r = true;
-        if (pt == 0)
-          r = mbar_wait(bar(V_FULL), seq & 1, vabort, kTimeoutNs) &&
-              mbar_wait(bar(XFREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
+        if (pt == 0) {
+          r = mbar_wait(bar(V_FULL), seq & 1, vabort, kTimeoutNs);
+          if (!F8) r = r && mbar_wait(bar(XFREE), (seq & 1) ^ 1, vabort, kTimeoutNs);
+        }
         if (!role_and(BAR_PREP, NP, r)) break;
       }
       if (F8) {
@@ -899,7 +902,10 @@ gdn_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      if (F8 || n < C) {
+      if (F8) {
+        fence_proxy_async_smem();
+        if (!wait_r(bar(XFREE), (seq & 1) ^ 1)) break;
+      } else if (n < C) {
         fence_proxy_async_smem();
         role_sync(BAR_PREP, NP);
       }
