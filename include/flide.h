@@ -291,7 +291,9 @@ int flide_quantize_e4m3(const void *x, int64_t n, int32_t dtype, const float *am
  *     FLIDE_ERR_CAPACITY before any work is queued.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture that should contain it.
+ *     before any stream capture that should contain it.  The address is then
+ *     kept for the life of the process: a cudaDeviceReset between calls is not
+ *     supported (the kept address would belong to the destroyed context).
  *   - All calls on a device share the one array.  Each call writes every entry
  *     it reads before reading it, so nothing needs clearing between calls, but
  *     calls whose executions overlap on the GPU (for example on two streams)
